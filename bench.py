@@ -1,0 +1,418 @@
+"""Benchmark of the packed-KV-cache per-layer step on B200.
+
+One step = one pass of the whole hot path for one layer of the pages-scale
+workload (B=1, 12 heads x 128, 6,240-token blocks, 40-block compressed pool,
+top-16, 27,872-key context):
+  select (query pooling + block scoring + top-k) -> attend -> append the
+  finished block (evicts the oldest compressed block) -> temporal RoPE shift
+  of the sink by 4 frames.
+Inputs are resident in HBM; L2 is flushed (256 MB write) between timed
+steps, outside the step's events.  The metric is packed-cache attention
+TFLOP/s (attention FLOPs of the step / step time) and the per-layer step
+latency; the roofline line is the attention kernel's own time.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+For N > 1 run under torchrun: every rank runs an independent replica (its
+own cache and stream of blocks, no data-path collective), time = max over
+ranks, value = the ranks' total work / that time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "layer"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+LAUNCHES_PER_STEP = 5          # qpool, score+top-k, attend, append copy, rope shift
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+def dist_env():
+    """(rank, world, local_rank) from torchrun's environment (1 process if absent)."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def dist_init(backend: str):
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world
+
+
+def reduce_max(x: float, device=None) -> float:
+    """Maximum of x over all ranks (x itself on one process)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.barrier()
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each replica draws its own blocks."""
+    return base + 7919 * rank
+
+
+# ---------------------------------------------------------------- helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def attention_flops(B, H, Lq, Lk, D=128) -> float:
+    """QK^T and PV: 2 multiply-adds per (query, key, dim), 2 FLOP each."""
+    return 4.0 * B * H * Lq * Lk * D
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def traffic_for(kernel_src: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current source of the kernel; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    ent = d.get(workload)
+    if not ent:
+        return None
+    with open(kernel_src, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()[:16]
+    return ent.get("dram_bytes_per_launch") if ent.get("source_sha") == h else None
+
+
+# ---------------------------------------------------------------- the GPU arm
+
+def run_gpu(args):
+    import torch
+
+    import synth
+    from packed_kv_cache_b200 import build as pfbuild
+    pfbuild.build()
+    import packed_kv_cache_b200 as pf
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dist_init("nccl")
+    dev = torch.device("cuda", local)
+    wl = synth.WORKLOADS[WORKLOAD]
+    B, H, D, n, nc = wl.batch, wl.heads, wl.head_dim, wl.n, wl.n_c
+    seed = rank_seed(synth.nominal_seed(list(synth.WORKLOADS).index(WORKLOAD)), rank)
+    d = synth.make_layer(wl, seed, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    cache = pf.PackedKVCache(pf.config_for(wl, layers=1), device=dev)
+    for s in range(wl.sink_blocks):
+        cache.append_block(0, d["sink_K"][:, s].contiguous(), d["sink_V"][:, s].contiguous())
+    cache.load_mid(0, d["mid_K"].contiguous(), d["mid_V"].contiguous())
+    for r in range(wl.recent_blocks):
+        cache.append_block(0, d["recent_K"][:, r].contiguous(), d["recent_V"][:, r].contiguous(),
+                           d["recent_Kc"][:, r].contiguous(), d["recent_Vc"][:, r].contiguous())
+    # the current block's inputs (resident); its compressed copy for the append
+    Q, Kn, Vn = d["Q"], d["K_cur"], d["V_cur"]
+    Kcn = synth.bf16_normal((B, nc, H, D), seed + 1, dev)
+    Vcn = synth.bf16_normal((B, nc, H, D), seed + 2, dev)
+    O = torch.empty_like(Q)
+    info0 = cache.info(0)
+    Lk = info0["context_tokens"]
+    flops = attention_flops(B, H, n, Lk, D)
+
+    ev_att = []
+
+    def step(q, k, v, kc, vc, out, att_events=None):
+        cache.select_mid(0, q)
+        if att_events is not None:
+            att_events[0].record(stream)
+        cache.attend(0, q, k, v, out)
+        if att_events is not None:
+            att_events[1].record(stream)
+        ev = cache.append_block(0, k, v, kc, vc)
+        if ev:
+            cache.rope_shift(0, pf.PART_SINK, ev * wl.block_frames)
+
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        step(Q, Kn, Vn, Kcn, Vcn, O)
+    torch.cuda.synchronize(dev)
+    cache.poll_device_error()
+    assert cache.info(0)["context_tokens"] == Lk
+
+    clocks = ClockSampler(local)
+    ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    ev_att = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks.start()
+    for i in range(args.steps):
+        flush.fill_((i + 7) & 0xFF)
+        ev_step[i][0].record(stream)
+        step(Q, Kn, Vn, Kcn, Vcn, O, ev_att[i])
+        ev_step[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    cache.poll_device_error()
+    step_ms = [a.elapsed_time(b) for a, b in ev_step]
+    att_ms = [a.elapsed_time(b) for a, b in ev_att]
+    total_ms = reduce_max(sum(step_ms), dev)
+    att_mean_ms = reduce_max(statistics.mean(att_ms), dev)
+    ms_per_step = total_ms / args.steps
+    value = world * args.steps * flops / (total_ms * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers
+    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+    hQ, hK, hV, hKc, hVc = pin(Q), pin(Kn), pin(Vn), pin(Kcn), pin(Vcn)
+    hO = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+    dQ, dK, dV, dKc, dVc = (torch.empty_like(t) for t in (Q, Kn, Vn, Kcn, Vcn))
+    h2d = sum(t.numel() * t.element_size() for t in (hQ, hK, hV, hKc, hVc))
+    d2h = hO.numel() * hO.element_size()
+
+    def e2e_step():
+        for dst, src in ((dQ, hQ), (dK, hK), (dV, hV), (dKc, hKc), (dVc, hVc)):
+            dst.copy_(src, non_blocking=True)
+        step(dQ, dK, dV, dKc, dVc, O)
+        hO.copy_(O, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = reduce_max(e0.elapsed_time(e1), dev)
+    e2e_value = world * args.steps * flops / (e2e_ms * 1e-3) / 1e12
+    cache.poll_device_error()
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = flops / (att_mean_ms * 1e-3) / 1e12
+    line = {
+        "metric": "packed-cache attention TFLOP/s (per-layer step)",
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": ("one layer, pages scale: B=1, H=12, d_h=128, block 4x30x52 (n=6240), "
+                         "compressed 182 tokens/block, pool 40, top-16, context 27872 keys; "
+                         "step = select + attend + append(evict) + sink RoPE shift"),
+            "context_tokens": Lk,
+            "attention_flop_per_step": flops,
+            "l2": "flushed between steps (256 MB write), outside the step events",
+            "parallelism": f"replicas x{world} (independent streams, no collective)",
+        },
+        "attention_ms": round(att_mean_ms, 4),
+        "roofline": {
+            "kernel": "attend_kernel",
+            "bound": "tensor",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4),
+            "peak_source": f"{peak_src} bf16 dense (burst)",
+            "traffic": traffic_for(os.path.join(ROOT, "packed_kv_cache_b200", "csrc", "attend.cu"), WORKLOAD),
+        },
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / args.steps, 4)},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(d, wl, budget_s=args.cpu_seconds)
+    cache.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------- the oracle on host cores
+
+def oracle_step(d, wl, rows):
+    """One bounded sample of the step on the CPU oracle: selection over the
+    whole pool, the sink shift, and attention for ``rows`` query rows."""
+    import oracle
+    S = oracle.select_scores(d["Q"], d["mid_K"])
+    sel = oracle.select_topk(S, wl.n_top)
+    B, H, D = wl.batch, wl.heads, wl.head_dim
+    sinkK = oracle.rope_shift(d["sink_K"].reshape(B, -1, H, D), wl.block_frames)
+    parts = [(sinkK, d["sink_V"].reshape(B, -1, H, D))]
+    mK = [oracle.to_f64(d["mid_K"][b, sel[b]]).reshape(-1, H, D) for b in range(B)]
+    mV = [oracle.to_f64(d["mid_V"][b, sel[b]]).reshape(-1, H, D) for b in range(B)]
+    import numpy as np
+    parts.append((np.stack(mK), np.stack(mV)))
+    parts.append((d["recent_K"].reshape(B, -1, H, D), d["recent_V"].reshape(B, -1, H, D)))
+    parts.append((d["K_cur"], d["V_cur"]))
+    oracle.attend(d["Q"], parts, rows=rows)
+    Lk = sum(p[0].shape[1] for p in parts)
+    return attention_flops(B, H, len(rows), Lk, D)
+
+
+def cpu_baseline(d, wl, budget_s=15.0):
+    import numpy as np
+    dc = {k: (v.cpu() if hasattr(v, "cpu") else v) for k, v in d.items()}
+    rows = np.arange(16)
+    t0 = time.perf_counter()
+    fl = oracle_step(dc, wl, rows)
+    dt = time.perf_counter() - t0
+    # grow the sample toward the budget
+    nrows = int(min(wl.n, max(16, 16 * budget_s / max(dt, 1e-3) * 0.8)))
+    rows = np.linspace(0, wl.n - 1, nrows).astype(np.int64)
+    t0 = time.perf_counter()
+    fl = oracle_step(dc, wl, rows)
+    dt = time.perf_counter() - t0
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": (f"selection over the whole 40-block pool, sink RoPE shift, and attention of "
+                       f"{nrows} of 6240 query rows x 12 heads over the 27872-key context, float64 numpy; "
+                       f"{dt:.1f} s"), "seconds": round(dt, 2)}
+
+
+def run_reference(args):
+    import numpy as np
+
+    import synth
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    wl = synth.WORKLOADS[WORKLOAD]
+    d = synth.make_layer(wl, synth.nominal_seed(list(synth.WORKLOADS).index(WORKLOAD)))
+    rows = np.linspace(0, wl.n - 1, args.ref_rows).astype(np.int64)
+    for _ in range(args.warmup):
+        oracle_step(d, wl, rows)
+    t0 = time.perf_counter()
+    fl = 0.0
+    for _ in range(args.steps):
+        fl += oracle_step(d, wl, rows)
+    dt = time.perf_counter() - t0
+    v = fl / dt / 1e12
+    line = {
+        "impl": "reference",
+        "metric": "packed-cache attention TFLOP/s (per-layer step)",
+        "value": v, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": ("one layer, pages scale: B=1, H=12, d_h=128, n=6240, pool 40x182, "
+                                "top-16, context 27872 keys; oracle sample per step"),
+                   "rows_per_step": int(args.ref_rows)},
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": f"per step: selection over the whole pool, sink shift, attention of "
+                                   f"{args.ref_rows} of 6240 query rows x 12 heads"},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--ref-rows", type=int, default=24)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)   # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,228 @@
+/*
+ * pf.h -- C ABI of the packed KV cache for block-autoregressive video
+ * diffusion (PackForcing), single GPU, sm_100a.
+ *
+ * The cache of one transformer layer has three partitions (PackForcing
+ * (arXiv), "Sink Tokens", "Compressed Mid Tokens", "Recent & Current
+ * Tokens"):
+ *   sink    the first N_sink/B_f blocks at full resolution, never evicted;
+ *   mid     a ring ("pool") of compressed blocks, n_c tokens each, of which
+ *           the top N_top by query-key affinity are routed into attention;
+ *   recent  the last N_recent/B_f finished blocks at full resolution.
+ * The current block's K/V are passed to each attention call.  The attended
+ * context is sink || selected mid (oldest first) || recent || current
+ * ("Bounded Attention Context").
+ *
+ * Conventions for every entry point:
+ *  - Tensors are device pointers to contiguous bf16 in token-major layout
+ *    [B, L, H, D] (D = 128 innermost), 16-byte aligned.  "Kc/Vc" are the
+ *    compressed keys/values of one block, [B, n_c, H, D].
+ *  - The caller owns every device buffer, including the cache arena
+ *    (sized by pf_cache_bytes).  The library owns a small host struct.
+ *  - Every call is asynchronous on the caller's CUDA stream (passed as
+ *    void*, a cudaStream_t; NULL = the legacy default stream) and does not
+ *    synchronise the host, except pf_poll_device_error.  Calls on one cache
+ *    must be ordered on one stream: they share per-layer scratch memory in
+ *    the arena.
+ *  - Errors are return codes; pf_last_error() gives the calling thread's
+ *    last message.  A failed call leaves the cache state unchanged.
+ *  - Device-side failures (a bounded wait that gave up) are recorded in a
+ *    word in the arena; pf_poll_device_error reads and clears it.
+ */
+#ifndef PF_H
+#define PF_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pf_status {
+  PF_OK = 0,
+  PF_ERR_ARG = 1,         /* null/misaligned pointer, value out of range */
+  PF_ERR_ARENA = 2,       /* arena too small or not 256-byte aligned */
+  PF_ERR_STATE = 3,       /* call not valid in the cache's current state */
+  PF_ERR_CAPACITY = 4,    /* a size exceeds a configured or built-in limit */
+  PF_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed */
+  PF_ERR_TIMEOUT = 6,     /* a device-side bounded wait gave up */
+  PF_ERR_UNSUPPORTED = 7  /* configuration outside what the kernels support */
+} pf_status;
+
+/* partition mask bits for pf_rope_shift */
+#define PF_PART_SINK 1u
+#define PF_PART_MID 2u     /* live compressed blocks of the pool */
+#define PF_PART_RECENT 4u  /* recent full-res blocks and their pending compressed copies */
+
+typedef struct pf_config {
+  int layers;        /* transformer layers; each has its own cache */
+  int batch;         /* B: independent sequences sharing the call (e.g. CFG cond/uncond) */
+  int heads;         /* H (12 for Wan2.1-1.3B) */
+  int head_dim;      /* d_h; only 128 is supported */
+  int block_frames;  /* B_f latent frames per block (4) */
+  int h, w;          /* patches per frame after patchification (30 x 52) */
+  int sink_blocks;   /* N_sink / B_f (2); may be 0 */
+  int recent_blocks; /* N_recent / B_f (1); >= 1 */
+  int mid_capacity;  /* compressed blocks the pool keeps before evicting the oldest */
+  int n_top;         /* N_top: mid blocks routed into attention (16) */
+  int rope_split[3]; /* rotary dims per axis (temporal, height, width) = 44, 42, 42 */
+  float rope_base;   /* rotary base (10000) */
+} pf_config;
+
+typedef struct pf_cache pf_cache;
+
+typedef struct pf_layer_info {
+  int blocks_seen;       /* blocks appended to this layer so far */
+  int sink_filled;       /* sink blocks stored (<= sink_blocks) */
+  int recent_count;      /* recent blocks stored (<= recent_blocks) */
+  int recent_head;       /* recent ring slot of the oldest recent block */
+  int mid_count;         /* live compressed blocks in the pool */
+  int mid_head;          /* pool slot of the oldest live compressed block */
+  int pool_slots;        /* mid_capacity + recent_blocks */
+  int selection_valid;   /* 1 if a selection for the current pool is stored */
+  int n_selected;        /* mid blocks that pf_attend will route now */
+  int context_tokens;    /* keys pf_attend attends to now, current block included */
+  long long evicted;     /* compressed blocks evicted so far */
+  long long total_shift; /* sum of the temporal shifts applied to the sink, frames */
+  void* sink_k;          /* [B, sink_blocks*n, H, D] */
+  void* sink_v;
+  void* pool_k;          /* [B, pool_slots, n_c, H, D], ring */
+  void* pool_v;
+  void* recent_k;        /* [B, recent_blocks, n, H, D], ring */
+  void* recent_v;
+  int32_t* selection;    /* device [B, n_top]: pool slots of the stored selection */
+  float* scores;         /* device [B, pool_slots]: last block scores, by age (oldest first) */
+} pf_layer_info;
+
+/* Library version, e.g. 100 for 0.1.0. */
+int pf_version(void);
+
+/* Message of the calling thread's last failed call ("" if none). */
+const char* pf_last_error(void);
+
+/* Name of a status code. */
+const char* pf_status_string(pf_status s);
+
+/*
+ * Bytes of device memory a cache with this configuration needs: the three
+ * partitions of every layer plus per-layer selection scratch.  Token counts
+ * follow PackForcing (arXiv), "KV Caching" (n = B_f h w) and "Compressed Mid
+ * Tokens" (n_c = floor(B_f/2) floor(h/4) floor(w/4)).
+ * Errors: PF_ERR_ARG for a null pointer or a non-positive size,
+ * PF_ERR_UNSUPPORTED for head_dim != 128 or rope_split not summing to it.
+ */
+pf_status pf_cache_bytes(const pf_config* cfg, size_t* bytes);
+
+/*
+ * Create a cache over a caller-owned arena of at least pf_cache_bytes bytes,
+ * 256-byte aligned.  Zeroes the arena on `stream` (asynchronously).  The
+ * arena must outlive the cache; pf_cache_destroy frees only host state.
+ * Errors: PF_ERR_ARG, PF_ERR_ARENA (too small / misaligned), PF_ERR_UNSUPPORTED,
+ * PF_ERR_CUDA.
+ */
+pf_status pf_cache_create(const pf_config* cfg, void* dev_arena, size_t arena_bytes,
+                          void* stream, pf_cache** out);
+
+pf_status pf_cache_destroy(pf_cache* cache);
+
+/* Host-side snapshot of one layer's state and its device addresses. */
+pf_status pf_cache_layer_info(const pf_cache* cache, int layer, pf_layer_info* out);
+
+/*
+ * Append the block that has just been generated (PackForcing (arXiv),
+ * "Dual-Resolution Shifting Mechanism"; "The Position Misalignment Problem").
+ * K, V: [B, n, H, D], the block's full-resolution keys (already carrying
+ * their RoPE rotation) and values.  Kc, Vc: [B, n_c, H, D], the compressed
+ * copy computed alongside it.
+ *  - While the sink is not full, the block is stored in the sink; Kc/Vc are
+ *    ignored and may be NULL.
+ *  - Otherwise the block becomes the newest recent block and Kc/Vc are kept
+ *    with it; if the recent partition was full, its oldest block leaves it
+ *    and that block's compressed copy joins the mid pool; if the pool then
+ *    holds more than mid_capacity blocks, the oldest is evicted.
+ * *evicted (optional) receives the number of compressed blocks evicted by
+ * this call (0 or 1).  The caller then shifts the sink's temporal RoPE by
+ * delta = evicted * B_f frames (pf_rope_shift).  Invalidates the layer's
+ * stored selection if the pool changed.  One kernel launch.
+ */
+pf_status pf_cache_append_block(pf_cache* cache, int layer, const void* K, const void* V,
+                                const void* Kc, const void* Vc, int* evicted, void* stream);
+
+/*
+ * Push `nblocks` compressed blocks straight into the mid pool, oldest
+ * first, as if each had aged out of the recent partition: restoring a saved
+ * cache, or building a long history without the full-resolution blocks.
+ * Kc, Vc: [B, nblocks, n_c, H, D].  The sink must be full.  *evicted
+ * (optional) receives the number of blocks evicted.  One kernel launch.
+ */
+pf_status pf_cache_load_mid(pf_cache* cache, int layer, const void* Kc, const void* Vc,
+                            int nblocks, int* evicted, void* stream);
+
+/*
+ * Dynamic context selection (PackForcing digest, method step (3);
+ * PackForcing (arXiv), "Compressed Mid Tokens"): score every live
+ * compressed block of the layer's pool against the current block's queries,
+ *   S[b, p] = (1/H) sum_h qbar_{b,h} . kbar_{b,p,h} / sqrt(d_h),
+ * qbar / kbar the mean query of the current block and the mean key of block
+ * p, per head; then keep the n_top largest (ties to the older block).  The
+ * selection is stored in the arena for the layer's later pf_attend calls
+ * (selection runs at a block's first denoising step; the other steps reuse
+ * it).  Q: [B, n, H, D].
+ * sel_out (optional, device, [B, min(n_top, mid_count)] int32): the chosen
+ * blocks by age (0 = oldest live block), ascending.
+ * scores_out (optional, device, [B, mid_count] float): S by age.
+ * Two kernel launches; no host synchronisation.
+ */
+pf_status pf_select_mid(pf_cache* cache, int layer, const void* Q, int32_t* sel_out,
+                        float* scores_out, void* stream);
+
+/*
+ * Incremental temporal RoPE adjustment (PackForcing (arXiv), "Incremental
+ * RoPE adjustment"; digest, method step (4)): multiply the stored keys'
+ * temporal rotary pairs by e^{i theta_t,k delta},
+ *   (x_2k + i x_2k+1) <- (x_2k + i x_2k+1) e^{i theta_k delta},
+ *   theta_k = rope_base^(-2k / rope_split[0]),  k < rope_split[0] / 2,
+ * in float32, rounded to bf16 (nearest even), in place.  Height and width
+ * pairs and all values are left untouched.  `parts` is a mask of
+ * PF_PART_SINK / PF_PART_MID / PF_PART_RECENT; the method shifts the sink.
+ * layer = -1 shifts every layer.  delta is in latent frames (any sign).
+ * One kernel launch per layer.
+ */
+pf_status pf_rope_shift(pf_cache* cache, int layer, unsigned parts, int delta, void* stream);
+
+/*
+ * Attention of the current block's queries over the bounded context
+ * (PackForcing digest, KV-cache paragraph; PackForcing (arXiv), "Bounded
+ * Attention Context"):
+ *   O = softmax(Q K^T / sqrt(d_h)) V,  K/V = sink || selected mid || recent || current.
+ * No mask.  Q, K_cur, V_cur, O: [B, n, H, D] bf16; O must not alias the
+ * inputs.  lse (optional, device, [B, H, n] float): log-sum-exp of the
+ * scaled scores, natural log.  Mid blocks: the stored selection if valid;
+ * if the pool holds at most n_top blocks, all of them; otherwise
+ * PF_ERR_STATE (call pf_select_mid first).  One kernel launch (tcgen05
+ * tensor cores, TMA loads through the partitions in place).
+ */
+pf_status pf_attend(pf_cache* cache, int layer, const void* Q, const void* K_cur,
+                    const void* V_cur, void* O, float* lse, void* stream);
+
+/*
+ * Synchronise `stream`, then read and clear the cache's device error word.
+ * Returns PF_OK, or PF_ERR_TIMEOUT if a kernel's bounded wait gave up since
+ * the last poll.  *code (optional) receives the raw word (0 = none).
+ */
+pf_status pf_poll_device_error(pf_cache* cache, void* stream, unsigned* code);
+
+/*
+ * Self-test of the bounded device wait used by the kernels: one thread waits
+ * on a barrier that nothing completes, for about `timeout_us` microseconds,
+ * then records PF_ERR_TIMEOUT in the cache's error word and returns.  Lets
+ * a test check the timeout path without faulting or hanging the GPU.
+ */
+pf_status pf_selftest_wait_timeout(pf_cache* cache, unsigned timeout_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PF_H */

@@ -1,0 +1,250 @@
+"""Python binding of libpf, the packed-KV-cache C ABI (include/pf.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  PyTorch supplies device memory (the cache arena and the tensors)
+and the current CUDA stream.  Importing this package fails if the library has
+not been built (``python -m packed_kv_cache_b200.build``); there is no
+fallback.
+
+Functions keep the C names (``pf_cache_create``, ``pf_select_mid``, ...);
+``PackedKVCache`` wraps them for one cache.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "PFError", "Config", "LayerInfo", "PART_SINK", "PART_MID", "PART_RECENT",
+    "lib", "library_path", "pf_version", "pf_cache_bytes", "pf_cache_create", "pf_cache_destroy",
+    "pf_cache_layer_info", "pf_cache_append_block", "pf_cache_load_mid", "pf_select_mid",
+    "pf_rope_shift", "pf_attend", "pf_poll_device_error", "pf_selftest_wait_timeout",
+    "PackedKVCache", "config_for",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libpf.so")
+
+PART_SINK, PART_MID, PART_RECENT = 1, 2, 4
+STATUS = {0: "PF_OK", 1: "PF_ERR_ARG", 2: "PF_ERR_ARENA", 3: "PF_ERR_STATE", 4: "PF_ERR_CAPACITY",
+          5: "PF_ERR_CUDA", 6: "PF_ERR_TIMEOUT", 7: "PF_ERR_UNSUPPORTED"}
+
+
+class PFError(RuntimeError):
+    def __init__(self, func: str, status: int, message: str):
+        self.status = status
+        self.status_name = STATUS.get(status, str(status))
+        super().__init__(f"{func}: {self.status_name}: {message}")
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("layers", ctypes.c_int), ("batch", ctypes.c_int), ("heads", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("block_frames", ctypes.c_int), ("h", ctypes.c_int),
+                ("w", ctypes.c_int), ("sink_blocks", ctypes.c_int), ("recent_blocks", ctypes.c_int),
+                ("mid_capacity", ctypes.c_int), ("n_top", ctypes.c_int),
+                ("rope_split", ctypes.c_int * 3), ("rope_base", ctypes.c_float)]
+
+
+class LayerInfo(ctypes.Structure):
+    _fields_ = [("blocks_seen", ctypes.c_int), ("sink_filled", ctypes.c_int),
+                ("recent_count", ctypes.c_int), ("recent_head", ctypes.c_int),
+                ("mid_count", ctypes.c_int), ("mid_head", ctypes.c_int), ("pool_slots", ctypes.c_int),
+                ("selection_valid", ctypes.c_int), ("n_selected", ctypes.c_int),
+                ("context_tokens", ctypes.c_int), ("evicted", ctypes.c_longlong),
+                ("total_shift", ctypes.c_longlong),
+                ("sink_k", ctypes.c_void_p), ("sink_v", ctypes.c_void_p),
+                ("pool_k", ctypes.c_void_p), ("pool_v", ctypes.c_void_p),
+                ("recent_k", ctypes.c_void_p), ("recent_v", ctypes.c_void_p),
+                ("selection", ctypes.c_void_p), ("scores", ctypes.c_void_p)]
+
+    def as_dict(self) -> dict:
+        return {name: getattr(self, name) for name, _ in self._fields_}
+
+
+def _load():
+    if not os.path.exists(library_path):
+        raise ImportError(f"{library_path} is missing: build it with `python -m packed_kv_cache_b200.build`")
+    L = ctypes.CDLL(library_path)
+    vp, i32, u32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint
+    sig = {
+        "pf_version": ([], ctypes.c_int),
+        "pf_last_error": ([], ctypes.c_char_p),
+        "pf_status_string": ([i32], ctypes.c_char_p),
+        "pf_cache_bytes": ([ctypes.POINTER(Config), ctypes.POINTER(ctypes.c_size_t)], i32),
+        "pf_cache_create": ([ctypes.POINTER(Config), vp, ctypes.c_size_t, vp, ctypes.POINTER(vp)], i32),
+        "pf_cache_destroy": ([vp], i32),
+        "pf_cache_layer_info": ([vp, i32, ctypes.POINTER(LayerInfo)], i32),
+        "pf_cache_append_block": ([vp, i32, vp, vp, vp, vp, ctypes.POINTER(i32), vp], i32),
+        "pf_cache_load_mid": ([vp, i32, vp, vp, i32, ctypes.POINTER(i32), vp], i32),
+        "pf_select_mid": ([vp, i32, vp, vp, vp, vp], i32),
+        "pf_rope_shift": ([vp, i32, u32, i32, vp], i32),
+        "pf_attend": ([vp, i32, vp, vp, vp, vp, vp, vp], i32),
+        "pf_poll_device_error": ([vp, vp, ctypes.POINTER(u32)], i32),
+        "pf_selftest_wait_timeout": ([vp, u32, vp], i32),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    return L
+
+
+lib = _load()
+
+
+def _check(func: str, status: int) -> None:
+    if status != 0:
+        raise PFError(func, status, lib.pf_last_error().decode(errors="replace"))
+
+
+def _dev(t, name: str):
+    """Device address of a CUDA tensor (None stays None)."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        return int(t)
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def config_for(wl, layers: int | None = None) -> Config:
+    """A pf_config for a workload description (``synth.Workload`` or alike)."""
+    c = Config()
+    c.layers = layers if layers is not None else getattr(wl, "layers", 1)
+    c.batch, c.heads, c.head_dim = wl.batch, wl.heads, wl.head_dim
+    c.block_frames, c.h, c.w = wl.block_frames, wl.h, wl.w
+    c.sink_blocks, c.recent_blocks = wl.sink_blocks, wl.recent_blocks
+    c.mid_capacity, c.n_top = wl.mid_capacity, wl.n_top
+    c.rope_split[0], c.rope_split[1], c.rope_split[2] = wl.rope_split
+    c.rope_base = wl.rope_base
+    return c
+
+
+# ---------------------------------------------------------------- C-named calls
+
+def pf_version() -> int:
+    return lib.pf_version()
+
+
+def pf_cache_bytes(cfg: Config) -> int:
+    out = ctypes.c_size_t()
+    _check("pf_cache_bytes", lib.pf_cache_bytes(ctypes.byref(cfg), ctypes.byref(out)))
+    return out.value
+
+
+def pf_cache_create(cfg: Config, arena, arena_bytes: int | None = None, stream=None) -> ctypes.c_void_p:
+    ptr = _dev(arena, "arena")
+    nbytes = arena_bytes if arena_bytes is not None else arena.numel() * arena.element_size()
+    handle = ctypes.c_void_p()
+    _check("pf_cache_create", lib.pf_cache_create(ctypes.byref(cfg), ptr, nbytes, _stream(stream),
+                                                  ctypes.byref(handle)))
+    return handle
+
+
+def pf_cache_destroy(handle) -> None:
+    _check("pf_cache_destroy", lib.pf_cache_destroy(handle))
+
+
+def pf_cache_layer_info(handle, layer: int) -> dict:
+    info = LayerInfo()
+    _check("pf_cache_layer_info", lib.pf_cache_layer_info(handle, layer, ctypes.byref(info)))
+    return info.as_dict()
+
+
+def pf_cache_append_block(handle, layer, K, V, Kc=None, Vc=None, stream=None) -> int:
+    ev = ctypes.c_int(0)
+    _check("pf_cache_append_block", lib.pf_cache_append_block(
+        handle, layer, _dev(K, "K"), _dev(V, "V"), _dev(Kc, "Kc"), _dev(Vc, "Vc"), ctypes.byref(ev),
+        _stream(stream)))
+    return ev.value
+
+
+def pf_cache_load_mid(handle, layer, Kc, Vc, nblocks: int, stream=None) -> int:
+    ev = ctypes.c_int(0)
+    _check("pf_cache_load_mid", lib.pf_cache_load_mid(handle, layer, _dev(Kc, "Kc"), _dev(Vc, "Vc"),
+                                                      nblocks, ctypes.byref(ev), _stream(stream)))
+    return ev.value
+
+
+def pf_select_mid(handle, layer, Q, sel_out=None, scores_out=None, stream=None) -> None:
+    _check("pf_select_mid", lib.pf_select_mid(handle, layer, _dev(Q, "Q"), _dev(sel_out, "sel_out"),
+                                              _dev(scores_out, "scores_out"), _stream(stream)))
+
+
+def pf_rope_shift(handle, layer: int, parts: int, delta: int, stream=None) -> None:
+    _check("pf_rope_shift", lib.pf_rope_shift(handle, layer, parts, delta, _stream(stream)))
+
+
+def pf_attend(handle, layer, Q, K_cur, V_cur, O, lse=None, stream=None) -> None:
+    _check("pf_attend", lib.pf_attend(handle, layer, _dev(Q, "Q"), _dev(K_cur, "K_cur"), _dev(V_cur, "V_cur"),
+                                      _dev(O, "O"), _dev(lse, "lse"), _stream(stream)))
+
+
+def pf_poll_device_error(handle, stream=None) -> int:
+    code = ctypes.c_uint(0)
+    _check("pf_poll_device_error", lib.pf_poll_device_error(handle, _stream(stream), ctypes.byref(code)))
+    return code.value
+
+
+def pf_selftest_wait_timeout(handle, timeout_us: int, stream=None) -> None:
+    _check("pf_selftest_wait_timeout", lib.pf_selftest_wait_timeout(handle, timeout_us, _stream(stream)))
+
+
+# ---------------------------------------------------------------- one cache
+
+class PackedKVCache:
+    """A cache over a torch-allocated arena on one CUDA device."""
+
+    def __init__(self, cfg: Config, device="cuda", stream=None):
+        self.cfg = cfg
+        self.nbytes = pf_cache_bytes(cfg)
+        self.arena = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
+        self.handle = pf_cache_create(cfg, self.arena, self.nbytes, stream)
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            pf_cache_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def info(self, layer: int) -> dict:
+        return pf_cache_layer_info(self.handle, layer)
+
+    def append_block(self, layer, K, V, Kc=None, Vc=None, stream=None) -> int:
+        return pf_cache_append_block(self.handle, layer, K, V, Kc, Vc, stream)
+
+    def load_mid(self, layer, Kc, Vc, stream=None) -> int:
+        return pf_cache_load_mid(self.handle, layer, Kc, Vc, Kc.shape[1], stream)
+
+    def select_mid(self, layer, Q, sel_out=None, scores_out=None, stream=None) -> None:
+        pf_select_mid(self.handle, layer, Q, sel_out, scores_out, stream)
+
+    def rope_shift(self, layer, parts, delta, stream=None) -> None:
+        pf_rope_shift(self.handle, layer, parts, delta, stream)
+
+    def attend(self, layer, Q, K_cur, V_cur, O=None, lse=None, stream=None) -> torch.Tensor:
+        if O is None:
+            O = torch.empty_like(Q)
+        pf_attend(self.handle, layer, Q, K_cur, V_cur, O, lse, stream)
+        return O
+
+    def poll_device_error(self, stream=None) -> int:
+        return pf_poll_device_error(self.handle, stream)

@@ -1,0 +1,97 @@
+// pf_internal.h -- launch interfaces between the host state machine
+// (pf_cache.cpp) and the kernels.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace pf {
+
+constexpr int kHeadDim = 128;
+constexpr int kMaxSegs = 64;
+
+// Device error codes written to the cache's error word.
+constexpr unsigned kDevErrTimeoutBase = 0x100u;  // | site id
+
+// ------------------------------------------------------------- RoPE shift
+// A list of contiguous runs of "row-heads" (one head's 128-dim key vector,
+// 256 bytes), start[] = prefix sums of the run lengths.
+struct RowRuns {
+  int n;
+  long long start[kMaxSegs + 1];
+  void* ptr[kMaxSegs];
+};
+
+struct RopeTable {
+  int pairs;  // rotary pairs to rotate (rope_split[0] / 2)
+  float c[32];
+  float s[32];
+};
+
+cudaError_t launch_rope_shift(const RowRuns& runs, const RopeTable& tab, cudaStream_t st);
+
+// ------------------------------------------------------------- copies
+// start[] = prefix sums of run lengths in 16-byte units.
+struct CopyRuns {
+  int n;
+  long long start[kMaxSegs + 1];
+  void* dst[kMaxSegs];
+  const void* src[kMaxSegs];
+};
+
+cudaError_t launch_copy(const CopyRuns& runs, cudaStream_t st);
+
+// ------------------------------------------------------------- selection
+struct SelectArgs {
+  const void* Q;        // [B, n, H, D] bf16
+  int B, n, HD;         // HD = H * D
+  float* qsum;          // [B, HD] accumulator, zero on entry, left zero on exit
+  const void* pool_k;   // [B, slots, n_c, H, D] bf16
+  int slots, n_c;
+  int head, count;      // live blocks: age p -> slot (head + p) % slots
+  int chunk_rows;       // pool rows per scoring CTA
+  int chunks_per_block;
+  float score_scale;    // 1 / (n * n_c * H * sqrt(D))
+  float* partial;       // [B, slots, chunks_per_block]
+  float* scores;        // [B, slots] by age
+  unsigned* ticket;     // [B], zero on entry, left zero on exit
+  int n_top;
+  int32_t* sel_slots;   // [B, n_top] pool slots, ascending age
+  int32_t* sel_out;     // optional [B, k] ages
+  float* scores_out;    // optional [B, count]
+};
+
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
+
+// ------------------------------------------------------------- attention
+// Partition ids of the K/V tensor maps.
+enum { kPartSink = 0, kPartMid = 1, kPartRecent = 2, kPartCur = 3 };
+
+struct AttendParams {
+  CUtensorMap tm_q;     // Q  (D, H, n, B)
+  CUtensorMap tm_k[4];  // sink (D,H,S*n,B), mid (D,H,n_c,B*slots), recent (D,H,n,B*R), cur (D,H,n,B)
+  CUtensorMap tm_v[4];
+  void* O;              // [B, n, H, D] bf16
+  float* lse;           // optional [B, H, n]
+  int B, H, n, n_c;
+  int sink_rows;        // filled sink rows per batch item
+  int n_sel;            // mid blocks routed
+  const int32_t* sel_slots;  // [B, sel_stride] pool slots, or null: all live blocks
+  int sel_stride;
+  int mid_head, pool_slots;
+  int n_recent, recent_head, recent_slots;
+  int sb_sink, sb_mid, sb_blk;  // 32-row sub-boxes: sink total, per mid block, per full block
+  int n_sub, n_tiles;
+  int q_pairs;          // 256-query units per (b, h)
+  float scale_log2;     // log2(e) / sqrt(D)
+  unsigned* err;
+  long long timeout_cycles;
+};
+
+cudaError_t launch_attend(const AttendParams& p, cudaStream_t st);
+
+// ------------------------------------------------------------- self-test
+cudaError_t launch_wait_timeout_selftest(unsigned* err, long long timeout_cycles, cudaStream_t st);
+
+}  // namespace pf

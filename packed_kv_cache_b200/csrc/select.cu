@@ -1,0 +1,255 @@
+// select.cu -- dynamic top-k context selection over the compressed mid pool.
+//
+// PackForcing digest, method step (3): the affinity phi_j = sum_i q_i^T k_j
+// / sqrt(d) of the current block's queries with the compressed keys ranks
+// the mid blocks; the N_top best are routed into attention, the rest stay
+// archived (PackForcing (arXiv), "Compressed Mid Tokens").  Summed over a
+// block's keys and averaged over heads this is
+//   S[b, p] = sum_{j, h, d} qsum[b, h, d] * Kc[b, p, j, h, d] / (n n_c H sqrt(D)),
+// qsum = sum of the block's queries.  Two kernels, both HBM streams:
+//   1. qpool: 32-row chunks of Q summed per column, added into qsum[b].
+//   2. score: one CTA per 32-row chunk of a pool block, a dot product with
+//      qsum[b]; the last CTA of batch item b (ticket counter) sums the
+//      chunks of each block in a fixed order, runs an exact radix select of
+//      the n_top largest scores (ties to the older block), writes the
+//      selection in ascending age, and clears qsum[b] and its ticket.
+#include <cuda_bf16.h>
+
+#include "pf_internal.h"
+
+namespace pf {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ void acc_bf16x8(float* acc, const uint4& w) {
+  const uint32_t v[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&v[q]);
+    acc[2 * q] += __low2float(x);
+    acc[2 * q + 1] += __high2float(x);
+  }
+}
+
+__device__ __forceinline__ float dot_bf16x8(const uint4& w, const float* q) {
+  const uint32_t v[4] = {w.x, w.y, w.z, w.w};
+  float s = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&v[e]);
+    s = fmaf(__low2float(x), q[2 * e], s);
+    s = fmaf(__high2float(x), q[2 * e + 1], s);
+  }
+  return s;
+}
+
+// qsum[b, :] += column sums of Q rows [32 c, 32 c + 32) of batch item b.
+__global__ void __launch_bounds__(kThreads) qpool_kernel(const SelectArgs a) {
+  const int b = blockIdx.y;
+  const int G = a.HD / 8;                        // 16-byte groups per row
+  const int Gp = G < kThreads ? G : kThreads;    // groups handled per pass
+  const int rstep = kThreads / Gp;               // row phases per pass
+  const int t = threadIdx.x;
+  const int r0 = t / Gp, gl = t % Gp;
+  const int row_lo = blockIdx.x * 32;
+  const int row_hi = min(a.n, row_lo + 32);
+  __shared__ float red[kThreads * 8];
+  const uint4* Q = static_cast<const uint4*>(a.Q) + static_cast<long long>(b) * a.n * G;
+  for (int g0 = 0; g0 < G; g0 += Gp) {
+    const int g = g0 + gl;
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (r0 < rstep && g < G) {
+#pragma unroll 4
+      for (int r = row_lo + r0; r < row_hi; r += rstep) acc_bf16x8(acc, Q[static_cast<long long>(r) * G + g]);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[t * 8 + e] = acc[e];
+    __syncthreads();
+    if (r0 == 0 && g < G) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        float s = red[t * 8 + e];
+        for (int k = 1; k < rstep; ++k) s += red[(k * Gp + gl) * 8 + e];
+        atomicAdd(&a.qsum[static_cast<long long>(b) * a.HD + g * 8 + e], s);
+      }
+    }
+    __syncthreads();
+  }
+}
+
+__device__ __forceinline__ uint32_t order_key(float f) {
+  const uint32_t u = __float_as_uint(f + 0.0f);  // -0 -> +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// exclusive prefix sum over the block; returns this thread's offset, *total the sum
+__device__ unsigned block_exclusive_scan(unsigned v, unsigned* total) {
+  __shared__ unsigned warp_sums[kThreads / 32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  unsigned x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[w] = x;
+  __syncthreads();
+  unsigned before = 0, tot = 0;
+  for (int k = 0; k < kThreads / 32; ++k) {
+    if (k < w) before += warp_sums[k];
+    tot += warp_sums[k];
+  }
+  __syncthreads();
+  *total = tot;
+  return before + x - v;
+}
+
+__global__ void __launch_bounds__(kThreads) score_kernel(const SelectArgs a) {
+  extern __shared__ float smem[];
+  float* qs = smem;                                      // [HD]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + a.HD);  // [count]
+  __shared__ float red[kThreads / 32];
+  __shared__ unsigned is_last;
+  __shared__ unsigned hist[256];
+  __shared__ unsigned sh_prefix, sh_need;
+
+  const int b = blockIdx.y;
+  const int p = blockIdx.x / a.chunks_per_block;
+  const int c = blockIdx.x % a.chunks_per_block;
+  const int t = threadIdx.x;
+  const int G = a.HD / 8;
+
+  for (int i = t; i < a.HD; i += kThreads) qs[i] = a.qsum[static_cast<long long>(b) * a.HD + i];
+  __syncthreads();
+
+  const int slot = (a.head + p) % a.slots;
+  const int row_lo = c * a.chunk_rows;
+  const int rows = min(a.n_c, row_lo + a.chunk_rows) - row_lo;
+  const uint4* K = static_cast<const uint4*>(a.pool_k) +
+                   ((static_cast<long long>(b) * a.slots + slot) * a.n_c + row_lo) * G;
+  const int nu = rows * G;
+  float acc = 0.f;
+  constexpr int U = 8;
+  for (int u0 = t; u0 < nu; u0 += kThreads * U) {
+    uint4 w[U];
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      const int u = u0 + k * kThreads;
+      if (u < nu) w[k] = __ldg(K + u);
+    }
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      const int u = u0 + k * kThreads;
+      if (u < nu) acc += dot_bf16x8(w[k], qs + (u % G) * 8);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((t & 31) == 0) red[t >> 5] = acc;
+  __syncthreads();
+  if (t == 0) {
+    float s = 0.f;
+    for (int k = 0; k < kThreads / 32; ++k) s += red[k];
+    a.partial[(static_cast<long long>(b) * a.slots + p) * a.chunks_per_block + c] = s;
+    __threadfence();
+    const unsigned total = static_cast<unsigned>(a.count * a.chunks_per_block);
+    is_last = (atomicAdd(&a.ticket[b], 1u) == total - 1u) ? 1u : 0u;
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+
+  // ---- last CTA of batch item b: block scores, top-k, cleanup
+  const int count = a.count;
+  for (int q = t; q < count; q += kThreads) {
+    const float* pp = a.partial + (static_cast<long long>(b) * a.slots + q) * a.chunks_per_block;
+    float s = 0.f;
+    for (int k = 0; k < a.chunks_per_block; ++k) s += __ldcg(pp + k);
+    s *= a.score_scale;
+    keys[q] = order_key(s);
+    a.scores[static_cast<long long>(b) * a.slots + q] = s;
+    if (a.scores_out) a.scores_out[static_cast<long long>(b) * count + q] = s;
+  }
+  const int k_sel = min(a.n_top, count);
+  if (t == 0) {
+    sh_prefix = 0u;
+    sh_need = static_cast<unsigned>(k_sel);
+  }
+  __syncthreads();
+  const bool take_all = (k_sel == count);
+  if (!take_all) {
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      hist[t] = 0u;
+      __syncthreads();
+      const unsigned pre = sh_prefix;
+      for (int q = t; q < count; q += kThreads) {
+        const uint32_t key = keys[q];
+        if (shift == 24 || (key >> (shift + 8)) == (pre >> (shift + 8))) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      if (t == 0) {
+        unsigned cum = 0u;
+        for (int d = 255; d >= 0; --d) {
+          const unsigned hc = hist[d];
+          if (cum + hc >= sh_need) {
+            sh_prefix = pre | (static_cast<unsigned>(d) << shift);
+            sh_need -= cum;
+            break;
+          }
+          cum += hc;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  const uint32_t T = sh_prefix;
+  const unsigned need = sh_need;
+  const int per = (count + kThreads - 1) / kThreads;
+  const int lo = min(count, t * per), hi = min(count, lo + per);
+  // rank of each key equal to the threshold among the equal ones, by age
+  unsigned eqc = 0u, tot = 0u;
+  if (!take_all)
+    for (int q = lo; q < hi; ++q) eqc += (keys[q] == T) ? 1u : 0u;
+  const unsigned eq_before = block_exclusive_scan(eqc, &tot);
+  unsigned nsel = 0u, e = eq_before;
+  for (int q = lo; q < hi; ++q) {
+    const uint32_t key = keys[q];
+    const bool s = take_all || key > T || (key == T && e++ < need);
+    nsel += s ? 1u : 0u;
+  }
+  unsigned pos = block_exclusive_scan(nsel, &tot);
+  e = eq_before;
+  for (int q = lo; q < hi; ++q) {
+    const uint32_t key = keys[q];
+    const bool s = take_all || key > T || (key == T && e++ < need);
+    if (s) {
+      a.sel_slots[static_cast<long long>(b) * a.n_top + pos] = (a.head + q) % a.slots;
+      if (a.sel_out) a.sel_out[static_cast<long long>(b) * k_sel + pos] = q;
+      ++pos;
+    }
+  }
+  for (int i = t; i < a.HD; i += kThreads) a.qsum[static_cast<long long>(b) * a.HD + i] = 0.f;
+  if (t == 0) a.ticket[b] = 0u;
+}
+
+}  // namespace
+
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
+  if (a.count <= 0) return cudaSuccess;
+  dim3 g1((a.n + 31) / 32, a.B);
+  qpool_kernel<<<g1, kThreads, 0, st>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = static_cast<size_t>(a.HD) * 4 + static_cast<size_t>(a.count) * 4;
+  if (smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  dim3 g2(a.count * a.chunks_per_block, a.B);
+  score_kernel<<<g2, kThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace pf

@@ -1,0 +1,122 @@
+"""Host-only checks of the C-ABI library: it loads without a GPU, exports
+every function include/pf.h declares, sizes arenas and rejects bad
+arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pf.h")
+
+
+@pytest.fixture(scope="module")
+def pf():
+    from packed_kv_cache_b200 import build
+    build.build()
+    import packed_kv_cache_b200 as mod
+    return mod
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pf_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for want in ("pf_cache_bytes", "pf_cache_create", "pf_cache_destroy", "pf_cache_append_block",
+                 "pf_select_mid", "pf_rope_shift", "pf_attend", "pf_poll_device_error", "pf_last_error"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(pf):
+    lib = ctypes.CDLL(pf.library_path)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_version_and_status_strings(pf):
+    assert pf.pf_version() >= 100
+    assert pf.lib.pf_status_string(6) == b"PF_ERR_TIMEOUT"
+
+
+def _cfg(pf, **kw):
+    c = pf.config_for(synth.WORKLOADS["layer"])
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def test_cache_bytes_layout(pf):
+    wl = synth.WORKLOADS["layer"]
+    c = pf.config_for(wl)
+    got = pf.pf_cache_bytes(c)
+    row = 12 * 128 * 2
+    al = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    slots = wl.mid_capacity + wl.recent_blocks
+    cpb = (182 + 31) // 32
+    per_layer = (2 * (al(2 * 6240 * row) + al(slots * 182 * row) + al(6240 * row))
+                 + al(16 * 4) + al(slots * 4) + al(slots * cpb * 4) + al(12 * 128 * 4) + al(4))
+    assert got == 256 + per_layer
+    # layers scale linearly
+    c.layers = 30
+    assert pf.pf_cache_bytes(c) == 256 + 30 * per_layer
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("head_dim", 64, "PF_ERR_UNSUPPORTED"),
+    ("batch", 0, "PF_ERR_ARG"),
+    ("recent_blocks", 0, "PF_ERR_ARG"),
+    ("mid_capacity", 9000, "PF_ERR_CAPACITY"),
+    ("rope_base", 0.5, "PF_ERR_ARG"),
+])
+def test_config_validation(pf, field, value, status):
+    c = _cfg(pf, **{field: value})
+    with pytest.raises(pf.PFError) as e:
+        pf.pf_cache_bytes(c)
+    assert e.value.status_name == status
+
+
+def test_rope_split_validation(pf):
+    c = _cfg(pf)
+    c.rope_split[0] = 46
+    with pytest.raises(pf.PFError) as e:
+        pf.pf_cache_bytes(c)
+    assert e.value.status_name == "PF_ERR_UNSUPPORTED"
+
+
+def test_create_rejects_bad_arenas_before_device_work(pf):
+    c = _cfg(pf)
+    need = pf.pf_cache_bytes(c)
+    h = ctypes.c_void_p()
+    assert pf.lib.pf_cache_create(ctypes.byref(c), None, need, None, ctypes.byref(h)) == 1
+    assert pf.lib.pf_cache_create(ctypes.byref(c), 0x1000 + 16, need, None, ctypes.byref(h)) == 2
+    assert b"256-byte" in pf.lib.pf_last_error()
+    assert pf.lib.pf_cache_create(ctypes.byref(c), 0x100000, need - 1, None, ctypes.byref(h)) == 2
+    assert b"needed" in pf.lib.pf_last_error()
+
+
+def test_calls_reject_null_cache(pf):
+    assert pf.lib.pf_attend(None, 0, None, None, None, None, None, None) == 1
+    assert pf.lib.pf_select_mid(None, 0, None, None, None, None) == 1
+    assert pf.lib.pf_rope_shift(None, 0, 1, 4, None) == 1
+    assert pf.lib.pf_cache_destroy(None) == 1
+    assert pf.lib.pf_poll_device_error(None, None, None) == 1
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    # importing the binding from a copy without libpf.so must raise, not fall back
+    import shutil
+    import subprocess
+    import sys
+    pkg = tmp_path / "packed_kv_cache_b200"
+    pkg.mkdir()
+    shutil.copy(os.path.join(ROOT, "packed_kv_cache_b200", "__init__.py"), pkg / "__init__.py")
+    r = subprocess.run([sys.executable, "-c", "import packed_kv_cache_b200"], cwd=tmp_path,
+                       capture_output=True, text=True)
+    assert r.returncode != 0 and "libpf.so" in r.stderr

@@ -1,0 +1,375 @@
+"""GPU path vs the oracle, element by element, through the C ABI.
+
+Sizes: the small workloads are compared in full; the pages-scale ones on
+sampled query rows (first, last, ragged tail and random rows) at the shapes
+bench.py times.  Tolerances: selection bit-exact (inputs have a relative
+score margin >= 1e-3), attention max-abs 2e-2 and relative L2 5e-3, shifted
+keys 1e-2 (or one bf16 ulp) after rounding the oracle to bf16."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from _harness import (LSE_MAX_ABS, arena_view, assert_attention_close, assert_keys_close, build_cache,
+                      oracle_context, seed_for)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def pf():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from packed_kv_cache_b200 import build
+    build.build()
+    import packed_kv_cache_b200 as mod
+    return mod
+
+
+def _wl(name):
+    return synth.WORKLOADS[name]
+
+
+def _layer(name, device="cpu", with_values=True):
+    wl = _wl(name)
+    return wl, synth.make_layer(wl, seed_for(name), device=device, with_values=with_values)
+
+
+def _rows(n, k=48, seed=0):
+    g = np.random.default_rng(seed)
+    r = set([0, 1, 127, 128, 255, 256, n - 1, n - 2, n - 97, n - 96]) | set(g.integers(0, n, k).tolist())
+    return np.array(sorted(x for x in r if 0 <= x < n))
+
+
+# ------------------------------------------------------------------ RoPE shift
+
+@pytest.mark.parametrize("name", ["tiny", "ragged_a", "ragged_b", "layer"])
+def test_rope_shift_sink_matches_oracle(pf, name):
+    wl, d = _layer(name)
+    cache = build_cache(pf, wl, d)
+    info = cache.info(0)
+    B, S, n, H, D = wl.batch, wl.sink_blocks, wl.n, wl.heads, wl.head_dim
+    cache.rope_shift(0, pf.PART_SINK, d["delta"])
+    torch.cuda.synchronize()
+    got = arena_view(cache, info["sink_k"], (B, S * n, H, D)).cpu()
+    before = d["sink_K"].reshape(B, S * n, H, D)
+    ref = oracle.rope_shift(before, d["delta"])
+    assert_keys_close(got, ref, name)
+    assert torch.equal(got[..., 44:], before[..., 44:])
+    sv = arena_view(cache, info["sink_v"], (B, S * n, H, D)).cpu()
+    assert torch.equal(sv, d["sink_V"].reshape(B, S * n, H, D))
+    assert cache.info(0)["total_shift"] == d["delta"]
+
+
+def test_rope_shift_all_partitions_and_composition(pf):
+    wl, d = _layer("ragged_b")
+    cache = build_cache(pf, wl, d)
+    info = cache.info(0)
+    B, n, nc, H, D = wl.batch, wl.n, wl.n_c, wl.heads, wl.head_dim
+    parts = pf.PART_SINK | pf.PART_MID | pf.PART_RECENT
+    cache.rope_shift(0, parts, 7)
+    cache.rope_shift(0, parts, -3)
+    torch.cuda.synchronize()
+    slots = info["pool_slots"]
+    pool = arena_view(cache, info["pool_k"], (B, slots, nc, H, D)).cpu()
+    live = torch.stack([pool[:, (info["mid_head"] + p) % slots] for p in range(info["mid_count"])], 1)
+    # two shifts compose to one of 4 (each rounded to bf16 in between)
+    ref_mid = oracle.rope_shift(oracle.round_bf16(oracle.rope_shift(d["mid_K"], 7)), -3)
+    assert_keys_close(live, ref_mid, "mid")
+    rec = arena_view(cache, info["recent_k"], (B, wl.recent_blocks, n, H, D)).cpu()
+    rec = torch.stack([rec[:, (info["recent_head"] + r) % wl.recent_blocks] for r in range(info["recent_count"])], 1)
+    ref_rec = oracle.rope_shift(oracle.round_bf16(oracle.rope_shift(d["recent_K"], 7)), -3)
+    assert_keys_close(rec, ref_rec, "recent")
+    pend = torch.stack([pool[:, (info["mid_head"] + info["mid_count"] + r) % slots]
+                        for r in range(info["recent_count"])], 1)
+    ref_pend = oracle.rope_shift(oracle.round_bf16(oracle.rope_shift(d["recent_Kc"], 7)), -3)
+    assert_keys_close(pend, ref_pend, "pending compressed")
+
+
+def test_rope_shift_stress_full_size(pf):
+    # all cached keys of a batch-2, 1,000-block pool layer: sink + mid + recent
+    wl = _wl("stress16")
+    d = synth.make_layer(wl, seed_for("stress16"), device="cuda", with_values=False)
+    d["mid_V"] = torch.zeros_like(d["mid_K"])
+    d["sink_V"] = torch.zeros_like(d["sink_K"])
+    d["recent_V"] = torch.zeros_like(d["recent_K"])
+    cache = build_cache(pf, wl, d)
+    info = cache.info(0)
+    delta = d["delta"]
+    cache.rope_shift(0, pf.PART_SINK | pf.PART_MID | pf.PART_RECENT, delta)
+    torch.cuda.synchronize()
+    B, nc, H, D = wl.batch, wl.n_c, wl.heads, wl.head_dim
+    slots = info["pool_slots"]
+    pool = arena_view(cache, info["pool_k"], (B, slots, nc, H, D))
+    g = np.random.default_rng(1)
+    for p in sorted(g.choice(wl.pool_blocks, 24, replace=False).tolist()) + [0, wl.pool_blocks - 1]:
+        got = pool[:, (info["mid_head"] + p) % slots].cpu()
+        ref = oracle.rope_shift(d["mid_K"][:, p].cpu(), delta)
+        assert_keys_close(got, ref, f"mid block {p}")
+    sk = arena_view(cache, info["sink_k"], (B, 2 * wl.n, H, D))
+    rows = _rows(2 * wl.n)
+    assert_keys_close(sk[:, rows].cpu(), oracle.rope_shift(d["sink_K"].reshape(B, -1, H, D)[:, rows].cpu(), delta))
+
+
+# ------------------------------------------------------------------ selection
+
+@pytest.mark.parametrize("name", ["tiny", "ragged_a", "ragged_b", "layer", "step30", "stress16", "stress64"])
+def test_selection_bit_exact(pf, name):
+    wl = _wl(name)
+    d = synth.make_layer(wl, seed_for(name), device="cpu", with_values=False)
+    for k in ("mid_V", "sink_V", "recent_V"):
+        d[k] = torch.zeros_like(d[k.replace("V", "K")])
+    d["V_cur"] = torch.zeros_like(d["K_cur"])
+    cache = build_cache(pf, wl, d)
+    B, P = wl.batch, wl.pool_blocks
+    k = min(wl.n_top, P)
+    sel = torch.full((B, k), -1, dtype=torch.int32, device="cuda")
+    sc = torch.zeros((B, P), dtype=torch.float32, device="cuda")
+    Q = d["Q"].cuda()
+    cache.select_mid(0, Q, sel, sc)
+    torch.cuda.synchronize()
+    S_ref = oracle.select_scores(d["Q"], d["mid_K"])
+    sel_ref = oracle.select_topk(S_ref, wl.n_top)
+    assert np.all(oracle.selection_margin(S_ref, wl.n_top) >= 1e-3)
+    assert np.array_equal(sel.cpu().numpy(), sel_ref), name
+    assert np.array_equal(sel_ref, d["planted"].numpy())
+    scale = np.abs(S_ref).max(axis=1, keepdims=True)
+    assert np.max(np.abs(sc.cpu().numpy() - S_ref) / scale) < 1e-4
+    info = cache.info(0)
+    assert info["selection_valid"] == 1 and info["n_selected"] == k
+    # a second call on the same inputs gives the same answer (scratch is left clean)
+    sel2 = torch.full_like(sel, -1)
+    cache.select_mid(0, Q, sel2, None)
+    torch.cuda.synchronize()
+    assert torch.equal(sel, sel2)
+
+
+def test_selection_ties_go_to_older_blocks(pf):
+    wl = _wl("ragged_a").replace(pool_blocks=9, planted=0, mid_capacity=9, n_top=4)
+    d = synth.make_layer(wl, 5)
+    d["mid_K"] = torch.zeros_like(d["mid_K"])         # every score exactly 0
+    cache = build_cache(pf, wl, d)
+    sel = torch.full((wl.batch, 4), -1, dtype=torch.int32, device="cuda")
+    cache.select_mid(0, d["Q"].cuda(), sel, None)
+    torch.cuda.synchronize()
+    assert sel.cpu().tolist() == [[0, 1, 2, 3]] * wl.batch
+
+
+# ------------------------------------------------------------------ attention
+
+def _attend_and_compare(pf, wl, d, rows=None, via_append=False, lse_check=True):
+    cache = build_cache(pf, wl, d, via_append=via_append)
+    Q, Kc, Vc = d["Q"].cuda(), d["K_cur"].cuda(), d["V_cur"].cuda()
+    sel = None
+    if wl.pool_blocks:
+        k = min(wl.n_top, wl.pool_blocks)
+        s = torch.zeros((wl.batch, k), dtype=torch.int32, device="cuda")
+        cache.select_mid(0, Q, s, None)
+        sel = s.cpu().numpy()
+    lse = torch.zeros((wl.batch, wl.heads, wl.n), dtype=torch.float32, device="cuda")
+    O = cache.attend(0, Q, Kc, Vc, lse=lse)
+    assert cache.poll_device_error() == 0
+    O = O.cpu()
+    if sel is not None:
+        sel_ref = oracle.select_topk(oracle.select_scores(d["Q"], d["mid_K"]), wl.n_top)
+        assert np.array_equal(sel, sel_ref)
+    parts = oracle_context(wl, d, sel)
+    if rows is None:
+        O_ref, lse_ref = oracle.attend(d["Q"], parts)
+        res = assert_attention_close(O, O_ref, wl.name)
+        got_lse = lse.cpu().numpy()
+    else:
+        O_ref, lse_ref = oracle.attend(d["Q"], parts, rows=rows)
+        res = assert_attention_close(O[:, rows], O_ref, wl.name)
+        got_lse = lse.cpu().numpy()[:, :, rows]
+    if lse_check:
+        assert np.max(np.abs(got_lse - lse_ref)) < LSE_MAX_ABS
+    info = cache.info(0)
+    tc = oracle.token_counts(wl.block_frames, wl.h, wl.w, wl.sink_blocks * wl.block_frames,
+                             wl.recent_blocks * wl.block_frames, min(wl.n_top, wl.pool_blocks))
+    assert info["context_tokens"] == tc["context"]
+    return res
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged_a", "ragged_b"])
+def test_attention_small_full(pf, name):
+    wl, d = _layer(name)
+    _attend_and_compare(pf, wl, d)
+
+
+def test_attention_pool_filled_by_appends(pf):
+    wl, d = _layer("ragged_a")
+    _attend_and_compare(pf, wl, d, via_append=True)
+
+
+def test_attention_pages_scale_layer(pf):
+    # Lq 6,240 x Lk 27,872, 12 heads: the configuration bench.py times
+    wl, d = _layer("layer")
+    _attend_and_compare(pf, wl, d, rows=_rows(wl.n))
+
+
+@pytest.mark.parametrize("name", ["stress16", "stress64"])
+def test_attention_stress(pf, name):
+    wl = _wl(name)
+    d = synth.make_layer(wl, seed_for(name), device="cpu")
+    _attend_and_compare(pf, wl, d, rows=_rows(wl.n, k=24))
+
+
+def test_attention_dense_long_context(pf):
+    # 748,800 full-resolution keys (no selection), sampled rows, head by head
+    wl = _wl("dense")
+    d = synth.make_layer(wl, seed_for("dense"), device="cuda")
+    cache = build_cache(pf, wl, d)
+    assert cache.info(0)["context_tokens"] == 748800
+    O = cache.attend(0, d["Q"], d["K_cur"], d["V_cur"])
+    assert cache.poll_device_error() == 0
+    rows = _rows(wl.n, k=8)
+    O = O[:, rows].cpu()
+    B, H, D = wl.batch, wl.heads, wl.head_dim
+    recK = d["recent_K"].reshape(B, -1, H, D)
+    recV = d["recent_V"].reshape(B, -1, H, D)
+    for h in (0, 5, 11):
+        parts = [(recK[:, :, h:h + 1].cpu(), recV[:, :, h:h + 1].cpu()),
+                 (d["K_cur"][:, :, h:h + 1].cpu(), d["V_cur"][:, :, h:h + 1].cpu())]
+        O_ref, _ = oracle.attend(d["Q"][:, rows][:, :, h:h + 1].cpu(), parts)
+        assert_attention_close(O[:, :, h:h + 1], O_ref, f"dense head {h}")
+
+
+def test_attention_early_blocks_partial_sink_empty_pool(pf):
+    wl = _wl("ragged_a")
+    d = synth.make_layer(wl, 11)
+    cache = pf.PackedKVCache(pf.config_for(wl, layers=1))
+    Q, Kc, Vc = d["Q"].cuda(), d["K_cur"].cuda(), d["V_cur"].cuda()
+    # no history at all: the block attends to itself
+    O = cache.attend(0, Q, Kc, Vc).cpu()
+    O_ref, _ = oracle.attend(d["Q"], [(d["K_cur"], d["V_cur"])])
+    assert_attention_close(O, O_ref, "empty cache")
+    # one of two sink blocks stored
+    cache.append_block(0, d["sink_K"][:, 0].cuda().contiguous(), d["sink_V"][:, 0].cuda().contiguous())
+    O = cache.attend(0, Q, Kc, Vc).cpu()
+    O_ref, _ = oracle.attend(d["Q"], [(d["sink_K"][:, 0], d["sink_V"][:, 0]), (d["K_cur"], d["V_cur"])])
+    assert_attention_close(O, O_ref, "half sink")
+
+
+def test_attention_needs_selection_when_pool_exceeds_n_top(pf):
+    wl, d = _layer("ragged_a")
+    cache = build_cache(pf, wl, d)
+    with pytest.raises(pf.PFError) as e:
+        cache.attend(0, d["Q"].cuda(), d["K_cur"].cuda(), d["V_cur"].cuda())
+    assert e.value.status_name == "PF_ERR_STATE"
+
+
+def test_attention_n_top_zero(pf):
+    wl = _wl("ragged_a").replace(n_top=0, planted=0)
+    d = synth.make_layer(wl, 3)
+    cache = build_cache(pf, wl, d)
+    cache.select_mid(0, d["Q"].cuda())
+    O = cache.attend(0, d["Q"].cuda(), d["K_cur"].cuda(), d["V_cur"].cuda()).cpu()
+    O_ref, _ = oracle.attend(d["Q"], oracle_context(wl, d, None))
+    assert_attention_close(O, O_ref, "n_top=0")
+
+
+# ------------------------------------------------------------------ cache state machine
+
+def test_state_machine_against_partition_model(pf):
+    wl = _wl("tiny").replace(mid_capacity=3, recent_blocks=2, n_top=2, planted=0, pool_blocks=0)
+    cfg = pf.config_for(wl, layers=2)
+    cache = pf.PackedKVCache(cfg)
+    B, n, nc, H, D = wl.batch, wl.n, wl.n_c, wl.heads, wl.head_dim
+    total_ev = 0
+    for i in range(10):
+        val = float(i + 1)
+        K = torch.full((B, n, H, D), val, dtype=torch.bfloat16, device="cuda")
+        Kc = torch.full((B, nc, H, D), val, dtype=torch.bfloat16, device="cuda")
+        ev = cache.append_block(1, K, K, Kc, Kc)
+        total_ev += ev
+        want = oracle.cache_partitions(i + 1, wl.sink_blocks, wl.recent_blocks, wl.mid_capacity)
+        info = cache.info(1)
+        assert info["sink_filled"] == len(want["sink"])
+        assert info["mid_count"] == len(want["mid"])
+        assert info["recent_count"] == len(want["recent"])
+        assert info["evicted"] == want["evicted"] == total_ev
+        torch.cuda.synchronize()
+        slots = info["pool_slots"]
+        pool = arena_view(cache, info["pool_k"], (B, slots, nc, H, D)).cpu()
+        got_mid = [pool[0, (info["mid_head"] + p) % slots, 0, 0, 0].item() - 1 for p in range(info["mid_count"])]
+        assert got_mid == want["mid"]
+        rec = arena_view(cache, info["recent_k"], (B, wl.recent_blocks, n, H, D)).cpu()
+        got_rec = [rec[0, (info["recent_head"] + r) % wl.recent_blocks, 0, 0, 0].item() - 1
+                   for r in range(info["recent_count"])]
+        assert got_rec == want["recent"]
+        sink = arena_view(cache, info["sink_k"], (B, wl.sink_blocks * n, H, D)).cpu()
+        for s in want["sink"]:
+            assert sink[0, s * n, 0, 0].item() - 1 == s
+    assert cache.info(0)["blocks_seen"] == 0   # the other layer is untouched
+
+
+# ------------------------------------------------------------------ generation loop
+
+def test_generation_loop_against_oracle_model(pf):
+    """select -> attend -> append -> shift over several blocks, with the
+    oracle keeping its own copy of every partition."""
+    wl = _wl("ragged_a").replace(mid_capacity=4, n_top=2, planted=0)
+    B, n, nc, H, D, Bf = wl.batch, wl.n, wl.n_c, wl.heads, wl.head_dim, wl.block_frames
+    cache = pf.PackedKVCache(pf.config_for(wl, layers=1))
+    sinkK, sinkV, mid, recent = [], [], [], []     # oracle's partitions (bf16-valued float64 / tensors)
+    for i in range(12):
+        blk = synth.make_block(wl, 7000 + i)
+        Q = synth.bf16_normal((B, n, H, D), 9000 + i)
+        # attention of block i over the cache as it stands
+        qd = Q.cuda()
+        sel = None
+        if len(mid) > wl.n_top:
+            s = torch.zeros((B, wl.n_top), dtype=torch.int32, device="cuda")
+            cache.select_mid(0, qd, s, None)
+            sel = s.cpu().numpy()
+            mK = torch.stack([torch.stack([m[0][b] for m in mid]) for b in range(B)], 1)
+            S_ref = oracle.select_scores(Q, mK.transpose(0, 1))
+            if np.all(oracle.selection_margin(S_ref, wl.n_top) >= 1e-3):
+                assert np.array_equal(sel, oracle.select_topk(S_ref, wl.n_top))
+        O = cache.attend(0, qd, blk["K"].cuda(), blk["V"].cuda()).cpu()
+        parts = [(torch.from_numpy(k), v) for k, v in zip(sinkK, sinkV)]
+        if mid:
+            chosen = [list(range(len(mid)))] * B if sel is None else sel.tolist()
+            for j in range(len(chosen[0])):
+                parts.append((torch.stack([mid[chosen[b][j]][0][b] for b in range(B)]),
+                              torch.stack([mid[chosen[b][j]][1][b] for b in range(B)])))
+        parts += [(r[0], r[1]) for r in recent]
+        parts.append((blk["K"], blk["V"]))
+        O_ref, _ = oracle.attend(Q, parts)
+        assert_attention_close(O, O_ref, f"block {i}")
+        # the block is final: append it, shift the sink on eviction
+        ev = cache.append_block(0, blk["K"].cuda(), blk["V"].cuda(), blk["Kc"].cuda(), blk["Vc"].cuda())
+        if len(sinkK) < wl.sink_blocks:
+            sinkK.append(oracle.to_f64(blk["K"]))
+            sinkV.append(blk["V"])
+        else:
+            recent.append((blk["K"], blk["V"], blk["Kc"], blk["Vc"]))
+            if len(recent) > wl.recent_blocks:
+                old = recent.pop(0)
+                mid.append((old[2], old[3]))
+                if len(mid) > wl.mid_capacity:
+                    mid.pop(0)
+                    assert ev == 1
+        if ev:
+            cache.rope_shift(0, pf.PART_SINK, ev * Bf)
+            sinkK = [oracle.round_bf16(oracle.rope_shift(k, ev * Bf)) for k in sinkK]
+    assert cache.info(0)["total_shift"] == cache.info(0)["evicted"] * Bf
+
+
+# ------------------------------------------------------------------ failure detection
+
+def test_bounded_wait_reports_timeout_and_context_survives(pf):
+    wl, d = _layer("tiny")
+    cache = build_cache(pf, wl, d)
+    pf.pf_selftest_wait_timeout(cache.handle, 2000)
+    with pytest.raises(pf.PFError) as e:
+        cache.poll_device_error()
+    assert e.value.status_name == "PF_ERR_TIMEOUT"
+    assert cache.poll_device_error() == 0          # cleared
+    # the device is still usable
+    cache.select_mid(0, d["Q"].cuda())
+    O = cache.attend(0, d["Q"].cuda(), d["K_cur"].cuda(), d["V_cur"].cuda())
+    torch.cuda.synchronize()
+    assert torch.isfinite(O.float()).all()
