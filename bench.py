@@ -95,7 +95,7 @@ def attention_flops(B, H, Lq, Lk, D=128) -> float:
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons during a region."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -114,7 +114,8 @@ class ClockSampler:
         except (OSError, FileNotFoundError):
             self.proc = None
 
-    def stop(self):
+    def stop(self, t0: float | None = None, t1: float | None = None):
+        """Stop sampling; summarise the samples taken between host times t0 and t1."""
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -122,12 +123,20 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
+        import datetime
         rows = []
         with open(self.path) as f:
             for line in f:
                 parts = [x.strip() for x in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
+                if len(parts) < 9:
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                except ValueError:
+                    ts = None
+                if t0 is not None and ts is not None and not (t0 <= ts <= t1):
+                    continue
+                rows.append(parts)
         os.unlink(self.path)
         if not rows:
             return None
@@ -209,6 +218,8 @@ def run_gpu(args):
         if ev:
             cache.rope_shift(0, pf.PART_SINK, ev * wl.block_frames)
 
+    clocks = ClockSampler(local)
+    clocks.start()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     for i in range(args.warmup):
         flush.fill_(i & 0xFF)
@@ -217,22 +228,22 @@ def run_gpu(args):
     cache.poll_device_error()
     assert cache.info(0)["context_tokens"] == Lk
 
-    clocks = ClockSampler(local)
     ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]
     ev_att = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
     torch.cuda.synchronize(dev)
     barrier()
-    clocks.start()
+    t_start = time.time()
     for i in range(args.steps):
         flush.fill_((i + 7) & 0xFF)
         ev_step[i][0].record(stream)
         step(Q, Kn, Vn, Kcn, Vcn, O, ev_att[i])
         ev_step[i][1].record(stream)
     torch.cuda.synchronize(dev)
+    t_end = time.time()
     barrier()
-    clk = clocks.stop()
+    clk = clocks.stop(t_start, t_end)
     cache.poll_device_error()
     step_ms = [a.elapsed_time(b) for a, b in ev_step]
     att_ms = [a.elapsed_time(b) for a, b in ev_att]
@@ -400,8 +411,8 @@ def run_reference(args):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--ref-rows", type=int, default=24)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

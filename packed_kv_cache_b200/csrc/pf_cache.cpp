@@ -620,11 +620,14 @@ pf_status pf_attend(pf_cache* c, int layer, const void* Q, const void* K_cur, co
   p.sb_blk = (g.n + 31) / 32;
   p.n_sub = p.sb_sink + n_sel * p.sb_mid + p.n_recent * p.sb_blk + p.sb_blk;
   p.n_tiles = (p.n_sub + 3) / 4;
-  p.q_pairs = (g.n + 255) / 256;
+  p.sb_mid_lo = p.sb_sink;
+  p.sb_mid_hi = p.sb_sink + n_sel * p.sb_mid;
+  p.exact = (sink_rows % 32 == 0 && g.n % 32 == 0) ? 1 : 0;
+  p.q_tiles = (g.n + 127) / 128;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
   p.err = c->err;
   p.timeout_cycles = c->timeout_cycles;
-  const long long units = 1LL * B * H * p.q_pairs;
+  const long long units = 1LL * B * H * p.q_tiles;
   if (units > 0x7fffffffLL) return fail(PF_ERR_CAPACITY, "too many work units");
   cudaError_t e = pf::launch_attend(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "attend launch");

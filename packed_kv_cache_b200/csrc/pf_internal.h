@@ -82,8 +82,11 @@ struct AttendParams {
   int mid_head, pool_slots;
   int n_recent, recent_head, recent_slots;
   int sb_sink, sb_mid, sb_blk;  // 32-row sub-boxes: sink total, per mid block, per full block
-  int n_sub, n_tiles;
-  int q_pairs;          // 256-query units per (b, h)
+  int n_sub, n_tiles;   // sub-boxes holding keys; 128-key tiles (n_sub padded to 4)
+  int sb_mid_lo, sb_mid_hi;  // sub-box range of the mid blocks
+  int exact;            // sink rows and block rows are multiples of 32: only mid blocks and
+                        // the padding after the last key have partial sub-boxes
+  int q_tiles;          // 128-row query tiles per (b, h)
   float scale_log2;     // log2(e) / sqrt(D)
   unsigned* err;
   long long timeout_cycles;
