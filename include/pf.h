@@ -207,6 +207,48 @@ pf_status pf_attend(pf_cache* cache, int layer, const void* Q, const void* K_cur
                     const void* V_cur, void* O, float* lse, void* stream);
 
 /*
+ * Limits of pf_select_mid_static (its scratch is a fixed array in the library).
+ */
+#define PF_STATIC_MAX_BATCH 8
+#define PF_STATIC_MAX_HEADS 16
+#define PF_STATIC_MAX_BLOCKS 4096
+#define PF_STATIC_MAX_NC 512
+
+/*
+ * The same block scoring and top-k selection as pf_select_mid, for callers
+ * that cannot allocate device memory for this library: a serving process
+ * that reserves its whole device-memory budget at start-up and allows no
+ * allocation on the request path (cudaMalloc and cudaFree can synchronise
+ * the device and fragment the pool), or a framework that owns the device
+ * allocator and passes only its own input and output tensors, with no cache
+ * arena.  This entry point allocates nothing: its scratch (query sums,
+ * partial and final block scores, the chosen slots, completion tickets) is
+ * one file-scope device array of about 2.4 MB, which every GPU that loads
+ * the library holds until the process exits.  (It has no counterpart on the
+ * pages; it is an interface choice of this library.)
+ *
+ * Q:       [batch, n, heads, 128] bf16, device, the current block's queries.
+ * pool_k:  [batch, pool_slots, n_c, heads, 128] bf16, device, a ring of
+ *          compressed keys; the live blocks, oldest first, are the slots
+ *          head, head+1, ... (mod pool_slots), `count` of them.
+ * sel_out: [batch, min(n_top, count)] int32, device: the chosen blocks by
+ *          age (0 = oldest live block), ascending.  Required.
+ * scores_out (optional): [batch, count] float, device: the block scores.
+ * Limits: batch <= PF_STATIC_MAX_BATCH, heads <= PF_STATIC_MAX_HEADS,
+ * count <= PF_STATIC_MAX_BLOCKS, n_c <= PF_STATIC_MAX_NC; larger sizes
+ * return PF_ERR_CAPACITY before any device work.
+ * The first call on a device looks up the array's device address with that
+ * device current (make that first call before any stream capture).  Every
+ * call clears what must start at zero and then shares the one array: calls
+ * that overlap on the GPU (different streams, or different host threads,
+ * on one device) race and must not be made.  Three launches on `stream`
+ * (one memset, two kernels); no host synchronisation.
+ */
+pf_status pf_select_mid_static(const void* Q, int batch, int n, int heads, const void* pool_k, int pool_slots,
+                               int n_c, int head, int count, int n_top, int32_t* sel_out, float* scores_out,
+                               void* stream);
+
+/*
  * Synchronise `stream`, then read and clear the cache's device error word.
  * Returns PF_OK, or PF_ERR_TIMEOUT if a kernel's bounded wait gave up since
  * the last poll.  *code (optional) receives the raw word (0 = none).

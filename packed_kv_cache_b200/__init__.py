@@ -21,6 +21,7 @@ __all__ = [
     "lib", "library_path", "pf_version", "pf_cache_bytes", "pf_cache_create", "pf_cache_destroy",
     "pf_cache_layer_info", "pf_cache_append_block", "pf_cache_load_mid", "pf_select_mid",
     "pf_rope_shift", "pf_attend", "pf_poll_device_error", "pf_selftest_wait_timeout",
+    "pf_select_mid_static",
     "PackedKVCache", "config_for",
 ]
 
@@ -83,6 +84,7 @@ def _load():
         "pf_attend": ([vp, i32, vp, vp, vp, vp, vp, vp], i32),
         "pf_poll_device_error": ([vp, vp, ctypes.POINTER(u32)], i32),
         "pf_selftest_wait_timeout": ([vp, u32, vp], i32),
+        "pf_select_mid_static": ([vp, i32, i32, i32, vp, i32, i32, i32, i32, i32, vp, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -201,6 +203,15 @@ def pf_poll_device_error(handle, stream=None) -> int:
 
 def pf_selftest_wait_timeout(handle, timeout_us: int, stream=None) -> None:
     _check("pf_selftest_wait_timeout", lib.pf_selftest_wait_timeout(handle, timeout_us, _stream(stream)))
+
+
+def pf_select_mid_static(Q, batch, n, heads, pool_k, pool_slots, n_c, head, count, n_top, sel_out,
+                         scores_out=None, stream=None) -> None:
+    """Selection with no device allocation (scratch in a fixed array inside
+    the library): for callers that cannot allocate device memory."""
+    _check("pf_select_mid_static", lib.pf_select_mid_static(
+        _dev(Q, "Q"), batch, n, heads, _dev(pool_k, "pool_k"), pool_slots, n_c, head, count, n_top,
+        _dev(sel_out, "sel_out"), _dev(scores_out, "scores_out"), _stream(stream)))
 
 
 # ---------------------------------------------------------------- one cache

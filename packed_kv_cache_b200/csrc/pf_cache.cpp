@@ -136,6 +136,18 @@ EncodeTiledFn get_encode_fn() {
 
 }  // namespace
 
+namespace pf {
+int report_error(int status, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return status;
+}
+}  // namespace pf
+
 struct pf_cache {
   pf_config cfg;
   Geometry g;

@@ -94,6 +94,9 @@ struct AttendParams {
 
 cudaError_t launch_attend(const AttendParams& p, cudaStream_t st);
 
+// Record a failure message for pf_last_error() and return the status.
+int report_error(int status, const char* fmt, ...);
+
 // ------------------------------------------------------------- self-test
 cudaError_t launch_wait_timeout_selftest(unsigned* err, long long timeout_cycles, cudaStream_t st);
 

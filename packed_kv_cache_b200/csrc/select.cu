@@ -15,6 +15,11 @@
 //      selection in ascending age, and clears qsum[b] and its ticket.
 #include <cuda_bf16.h>
 
+#include <cmath>
+#include <cstddef>
+#include <mutex>
+
+#include "pf.h"
 #include "pf_internal.h"
 
 namespace pf {
@@ -250,6 +255,123 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
   dim3 g2(a.count * a.chunks_per_block, a.B);
   score_kernel<<<g2, kThreads, smem, st>>>(a);
   return cudaGetLastError();
+}
+
+
+// ---------------------------------------------------------------------------
+// Selection with no device allocation.
+//
+// Some callers cannot allocate device memory for this library: a serving
+// process that reserves its whole device-memory budget at start-up and
+// forbids allocation on the request path (cudaMalloc/cudaFree can
+// synchronise the device and fragment the pool), or a host framework that
+// owns the device allocator and hands this code only its input and output
+// tensors, with no cache arena.  pf_select_mid_static serves them: the
+// selection's scratch (query sums, per-chunk partial scores, block scores,
+// slot list, tickets) lives in the file-scope array below, which every GPU
+// that loads the library holds until the process exits.
+namespace {
+
+constexpr int kStaticBatch = PF_STATIC_MAX_BATCH;
+constexpr int kStaticHD = PF_STATIC_MAX_HEADS * kHeadDim;
+constexpr int kStaticBlocks = PF_STATIC_MAX_BLOCKS;
+constexpr int kStaticChunks = (PF_STATIC_MAX_NC + 31) / 32;
+
+struct StaticSelectScratch {
+  float qsum[kStaticBatch * kStaticHD];
+  unsigned ticket[64];
+  float scores[kStaticBatch * kStaticBlocks];
+  int32_t sel_slots[kStaticBatch * kStaticBlocks];
+  float partial[kStaticBatch * kStaticBlocks * kStaticChunks];
+};
+
+static __device__ __align__(256) unsigned char g_select_scratch[sizeof(StaticSelectScratch)];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_select_scratch on the current device.  In host code
+// the array's name is a host-side stand-in, so the address is asked for once
+// per device, with that device current.
+cudaError_t static_scratch(StaticSelectScratch** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_select_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = p;
+  }
+  *out = static_cast<StaticSelectScratch*>(g_scratch_addr[dev]);
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" pf_status pf_select_mid_static(const void* Q, int batch, int n, int heads, const void* pool_k,
+                                          int pool_slots, int n_c, int head, int count, int n_top, int32_t* sel_out,
+                                          float* scores_out, void* stream) {
+  using pf::report_error;
+  if (Q == nullptr || pool_k == nullptr || sel_out == nullptr)
+    return static_cast<pf_status>(report_error(PF_ERR_ARG, "Q, pool_k and sel_out must not be NULL"));
+  if (reinterpret_cast<uintptr_t>(Q) % 16 != 0 || reinterpret_cast<uintptr_t>(pool_k) % 16 != 0 ||
+      reinterpret_cast<uintptr_t>(sel_out) % 4 != 0 ||
+      (scores_out != nullptr && reinterpret_cast<uintptr_t>(scores_out) % 4 != 0))
+    return static_cast<pf_status>(report_error(PF_ERR_ARG, "misaligned pointer"));
+  if (batch < 1 || n < 1 || heads < 1 || n_c < 1 || count < 0 || n_top < 0 || pool_slots < count ||
+      (pool_slots > 0 && (head < 0 || head >= pool_slots)))
+    return static_cast<pf_status>(report_error(PF_ERR_ARG, "bad sizes (batch %d, n %d, heads %d, n_c %d, "
+                                                            "slots %d, head %d, count %d, n_top %d)",
+                                               batch, n, heads, n_c, pool_slots, head, count, n_top));
+  if (batch > kStaticBatch || heads > PF_STATIC_MAX_HEADS || count > kStaticBlocks || n_c > PF_STATIC_MAX_NC)
+    return static_cast<pf_status>(report_error(
+        PF_ERR_CAPACITY, "pf_select_mid_static handles batch <= %d, heads <= %d, count <= %d, n_c <= %d",
+        kStaticBatch, PF_STATIC_MAX_HEADS, kStaticBlocks, PF_STATIC_MAX_NC));
+  // the kernels index partial[] and scores[] with the pool's slot count as stride
+  if (static_cast<long long>(batch) * pool_slots > kStaticBlocks * static_cast<long long>(kStaticBatch))
+    return static_cast<pf_status>(report_error(PF_ERR_CAPACITY, "batch * pool_slots must be <= %d",
+                                               kStaticBlocks * kStaticBatch));
+  if (count == 0 || n_top == 0) return PF_OK;
+  StaticSelectScratch* sc = nullptr;
+  cudaError_t e = static_scratch(&sc);
+  if (e != cudaSuccess)
+    return static_cast<pf_status>(report_error(PF_ERR_CUDA, "static scratch address: %s", cudaGetErrorString(e)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int HD = heads * kHeadDim;
+  // query sums and tickets must start at zero; they are contiguous
+  static_assert(offsetof(StaticSelectScratch, ticket) == sizeof(float) * kStaticBatch * kStaticHD, "layout");
+  e = cudaMemsetAsync(sc, 0, offsetof(StaticSelectScratch, scores), st);
+  if (e != cudaSuccess)
+    return static_cast<pf_status>(report_error(PF_ERR_CUDA, "clear static scratch: %s", cudaGetErrorString(e)));
+  SelectArgs a;
+  a.Q = Q;
+  a.B = batch;
+  a.n = n;
+  a.HD = HD;
+  a.qsum = sc->qsum;
+  a.pool_k = pool_k;
+  a.slots = pool_slots;
+  a.n_c = n_c;
+  a.head = head;
+  a.count = count;
+  a.chunk_rows = 32;
+  a.chunks_per_block = (n_c + 31) / 32;
+  a.score_scale = static_cast<float>(1.0 / (static_cast<double>(n) * n_c * heads * sqrt(128.0)));
+  a.partial = sc->partial;
+  a.scores = sc->scores;
+  a.ticket = sc->ticket;
+  a.n_top = n_top < count ? n_top : count;
+  a.sel_slots = sc->sel_slots;
+  a.sel_out = sel_out;
+  a.scores_out = scores_out;
+  e = launch_select(a, st);
+  if (e != cudaSuccess)
+    return static_cast<pf_status>(report_error(PF_ERR_CUDA, "select launch: %s", cudaGetErrorString(e)));
+  return PF_OK;
 }
 
 }  // namespace pf
