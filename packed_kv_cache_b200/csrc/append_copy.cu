@@ -3,7 +3,7 @@
 // Mechanism": the new full-resolution tokens replace the oldest recent
 // ones, the compressed copy is kept for when the block ages into the mid
 // partition).  All runs of one append go in a single launch; 16-byte
-// vectors, four loads in flight per thread, grid sized to the SM count.
+// vectors, four loads in flight per thread, grid = the CTAs resident at once.
 #include "pf_internal.h"
 
 namespace pf {
@@ -43,11 +43,16 @@ __global__ void __launch_bounds__(256) copy_runs_kernel(const CopyRuns runs) {
 cudaError_t launch_copy(const CopyRuns& runs, cudaStream_t st) {
   const long long total = runs.start[runs.n];
   if (total <= 0) return cudaSuccess;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  static int grid_cap = 0;
+  if (grid_cap == 0) {
+    int dev = 0, sms = 148, per_sm = 1;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, copy_runs_kernel, 256, 0);
+    grid_cap = sms * (per_sm > 0 ? per_sm : 1);
+  }
   const long long want = (total + 1023) / 1024;
-  const int grid = static_cast<int>(want < sms * 8LL ? want : sms * 8LL);
+  const int grid = static_cast<int>(want < grid_cap ? want : grid_cap);
   copy_runs_kernel<<<grid, 256, 0, st>>>(runs);
   return cudaGetLastError();
 }

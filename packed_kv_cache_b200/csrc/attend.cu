@@ -7,11 +7,17 @@
 // tokens.  The partitions are never gathered: the key/value tiles are pulled
 // by TMA straight from where each partition lives.
 //
-// Work unit: two 128-row query tiles of one (batch item, head) that share
-// every K/V tile, or the last, ragged tile of a (b, h) alone.  One CTA per
-// unit by default; a persistent grid (one CTA per SM, units dealt
-// round-robin) is available at build time.  12 warps:
-//   warp 0      TMA producer: Q per unit, K and V tiles through rings
+// Work units, one CTA each:
+//  * full unit: two 128-row query tiles of one (batch item, head) that share
+//    every K/V tile of the context;
+//  * tail chunk: when a block has an odd number of 128-row query tiles, the
+//    last (ragged) tile of each (b, h) is split along the context into k
+//    chunks of K/V tiles.  Each chunk writes its unnormalised output, row
+//    maximum and row sum to scratch; the chunk that finishes last merges them
+//    (O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c).  The chunks run after
+//    the full units and fill what would otherwise be a nearly idle last wave.
+// 12 warps per CTA:
+//   warp 0      TMA producer: Q, then K and V tiles through rings
 //   warp 1      MMA issuer (one thread): S_t = Q_t K^T and O_t += P_t V
 //   warp 2      tensor-memory allocator
 //   warps 4-7   softmax of query tile 0 (one thread per query row)
@@ -44,30 +50,21 @@ constexpr int kSub = 32;           // rows per TMA sub-box
 #define PF_ATTEND_K_STAGES 3
 #endif
 constexpr int kKStages = PF_ATTEND_K_STAGES;  // K ring depth
-constexpr int kVStages = 2;        // V ring depth
+constexpr int kVStages = 2;                   // V ring depth
 constexpr int kThreads = 384;
 constexpr uint32_t kTileBytes = kBN * kHeadDim * 2;   // 32 KB
 constexpr uint32_t kHalfBytes = kTileBytes / 2;       // 64 dims x 128 rows
 constexpr uint32_t kSubBytes = kSub * 128;            // one sub-box, one 64-dim half
 constexpr float kRescaleThreshold = 8.0f;
-// Registers per thread after the split: the producer/MMA warpgroup gives up
-// registers to the two softmax warpgroups (128*120 + 256*192 <= 384*168).
-#ifndef PF_ATTEND_REGS_CONTROL
-#define PF_ATTEND_REGS_CONTROL 120
-#endif
-#ifndef PF_ATTEND_REGS_SOFTMAX
-#define PF_ATTEND_REGS_SOFTMAX 192
-#endif
-constexpr int kRegsLaunch = 168, kRegsControl = PF_ATTEND_REGS_CONTROL, kRegsSoftmax = PF_ATTEND_REGS_SOFTMAX;
-static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
 // Before S_t of the next tile is written over P_t, wait until the P_t V MMA
-// that reads P_t has completed.
+// that reads P_t has completed.  Off by default: tcgen05.mma operations
+// issued by one thread execute in issue order.
 #ifndef PF_ATTEND_DRAIN
 #define PF_ATTEND_DRAIN 0
 #endif
 constexpr bool kDrainBeforeOverwrite = PF_ATTEND_DRAIN != 0;
 // One exponential pair in kPolyPeriod is evaluated by ex2_poly (FMA pipe),
-// the others by the special-function unit (0 = never).
+// the others by the special-function unit (0 = never; measured slower).
 #ifndef PF_ATTEND_POLY_PERIOD
 #define PF_ATTEND_POLY_PERIOD 0
 #endif
@@ -82,13 +79,14 @@ constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;           // + barriers + 
 static_assert(kSmemBytes <= 232448, "shared memory");
 
 struct Bars {
-  uint64_t q_full, q_empty;
+  uint64_t q_full;
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
-  uint64_t s_full[2], p_full[2], o_final[2], o_free[2];
+  uint64_t s_full[2], p_full[2], o_final[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  int merge;
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
 
@@ -146,74 +144,44 @@ __device__ __forceinline__ int subbox_valid(const AttendParams& p, int s) {
   return 0;
 }
 
-// One CTA per unit (1) or a persistent grid of at most one CTA per SM (0).
-// Measured on the pages-scale layer: 1.54 ms vs 1.74 ms.
-#ifndef PF_ATTEND_ONE_UNIT_PER_CTA
-#define PF_ATTEND_ONE_UNIT_PER_CTA 1
-#endif
-
-// The unit schedule.  A (b, h) has q_tiles 128-row query tiles.  Units
-// 0 .. F-1 pair tiles 2k and 2k+1 of one (b, h): both read the same K/V
-// tiles.  When q_tiles is odd, the last (ragged) tile of each (b, h) is a
-// unit of its own ("single").  Full units go round-robin over the G CTAs
-// (CTA c: c, c + G, ...), so that the CTAs running at the same time share
-// few heads; singles go round-robin over the CTAs that got fewer full units.
+// The unit of this CTA.  Units 0 .. F-1 are full units ((b, h) major, then
+// query-tile pair); then, if q_tiles is odd, B*H*tail_chunks tail chunks
+// ((b, h) major, then chunk).
 struct QTile {
   int b, h, qt;
 };
 struct Unit {
   QTile t[2];
   int nq;       // query tiles in the unit (1 or 2)
-  bool shared;  // both tiles read the same K/V stream
+  int j0, j1;   // K/V tiles [j0, j1) of the context
+  int tail;     // tail index ((b, h)) of a split tail, -1 otherwise
+  int chunk;    // chunk index within its tail
 };
-struct Sched {
-  int F, S, G, L0, NL;  // full units, singles, CTAs, first light CTA, light CTAs
-};
 
-__device__ __forceinline__ Sched make_sched(const AttendParams& p) {
-  Sched q;
-  q.F = p.B * p.H * (p.q_tiles / 2);
-  q.S = (p.q_tiles & 1) ? p.B * p.H : 0;
-  q.G = gridDim.x;
-  q.L0 = q.F % q.G;
-  q.NL = q.G - q.L0;
-  return q;
-}
-
-__device__ __forceinline__ int units_of(const Sched& q, int c) {
-#if PF_ATTEND_ONE_UNIT_PER_CTA
-  return c < q.F + q.S ? 1 : 0;
-#else
-  const int nf = q.F / q.G + (c < q.F % q.G ? 1 : 0);
-  const int ns = (c < q.L0 || q.S == 0) ? 0 : (q.S - (c - q.L0) + q.NL - 1) / q.NL;
-  return nf + max(ns, 0);
-#endif
-}
-
-__device__ __forceinline__ Unit unit_of(const AttendParams& p, const Sched& q, int c, int k) {
-#if PF_ATTEND_ONE_UNIT_PER_CTA
-  const int nf = c < q.F ? 1 : 0;
-  const int u = c;
-  (void)k;
-#else
-  const int nf = q.F / q.G + (c < q.F % q.G ? 1 : 0);
-  const int u = (k < nf) ? c + k * q.G : q.F + (c - q.L0) + (k - nf) * q.NL;
-#endif
+__device__ __forceinline__ Unit unit_of(const AttendParams& p, int u) {
   const int pairs = p.q_tiles / 2;
+  const int F = p.B * p.H * pairs;
   Unit r;
-  r.shared = true;
-  if (u < q.F) {
+  if (u < F) {
     const int bh = u / pairs, kk = u - bh * pairs;
     r.t[0] = {bh / p.H, bh % p.H, 2 * kk};
     r.t[1] = {bh / p.H, bh % p.H, 2 * kk + 1};
     r.nq = 2;
+    r.j0 = 0;
+    r.j1 = p.n_tiles;
+    r.tail = -1;
+    r.chunk = 0;
   } else {
-    const int bh = u - q.F;
+    const int v = u - F;
+    const int bh = v / p.tail_chunks, c = v - bh * p.tail_chunks;
     r.t[0] = {bh / p.H, bh % p.H, p.q_tiles - 1};
     r.t[1] = r.t[0];
     r.nq = 1;
+    r.j0 = static_cast<int>(static_cast<long long>(c) * p.n_tiles / p.tail_chunks);
+    r.j1 = static_cast<int>(static_cast<long long>(c + 1) * p.n_tiles / p.tail_chunks);
+    r.tail = (p.tail_chunks > 1) ? bh : -1;
+    r.chunk = c;
   }
-  (void)nf;
   return r;
 }
 
@@ -257,18 +225,20 @@ __device__ __forceinline__ void exp_chunk(const uint32_t* c, uint32_t dst, uint6
   tmem_st16(dst, pk);
 }
 
-#ifndef PF_ATTEND_SETMAXNREG
-#define PF_ATTEND_SETMAXNREG 0
-#endif
-__device__ __forceinline__ void setmaxnreg_dec() {
-#if PF_ATTEND_SETMAXNREG
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
-#endif
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
-__device__ __forceinline__ void setmaxnreg_inc() {
-#if PF_ATTEND_SETMAXNREG
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
-#endif
+
+__device__ __forceinline__ void store_row_bf16(uint4* dst, const float* o, float inv) {
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    uint4 w;
+    w.x = pack_bf16x2(o[8 * v + 0] * inv, o[8 * v + 1] * inv);
+    w.y = pack_bf16x2(o[8 * v + 2] * inv, o[8 * v + 3] * inv);
+    w.z = pack_bf16x2(o[8 * v + 4] * inv, o[8 * v + 5] * inv);
+    w.w = pack_bf16x2(o[8 * v + 6] * inv, o[8 * v + 7] * inv);
+    dst[v] = w;
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_constant__ AttendParams p) {
@@ -281,15 +251,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int T = p.n_tiles;
   const long long lim = p.timeout_cycles;
   volatile int* abort_flag = &bars.abort;
-  const Sched sched = make_sched(p);
-  const int n_units = units_of(sched, blockIdx.x);
+  const Unit un = unit_of(p, blockIdx.x);
+  const int nq = un.nq;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars.q_full, 1);
-    mbar_init(&bars.q_empty, 1);
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(&bars.k_full[s], 1);
       mbar_init(&bars.k_empty[s], 1);
@@ -302,10 +270,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
       mbar_init(&bars.s_full[t], 1);
       mbar_init(&bars.p_full[t], kBM);
       mbar_init(&bars.o_final[t], 1);
-      mbar_init(&bars.o_free[t], kBM);
     }
     mbar_init(&bars.drain, 1);
     bars.abort = 0;
+    bars.merge = 0;
     fence_mbar_init();
   }
   if (warp == 2) {
@@ -317,76 +285,68 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
 
-  if (warp < 4) {
-    setmaxnreg_dec();
-    if (warp == 0 && lane == 0) {
+  if (warp == 0) {
+    if (lane == 0) {
       // ---------------------------------------------------------- producer
       prefetch_tmap(&p.tm_q);
       for (int m = 0; m < 4; ++m) {
         prefetch_tmap(&p.tm_k[m]);
         prefetch_tmap(&p.tm_v[m]);
       }
-      int kg = 0, vg = 0;              // K / V tiles issued so far (all units)
-      int uq = 0;                      // units whose Q was loaded
+      mbar_arrive_expect_tx(&bars.q_full, nq * kTileBytes);
+      for (int t = 0; t < nq; ++t)
+        for (int half = 0; half < 2; ++half)
+          tma_load_4d(smem + kOffQ + t * kTileBytes + half * kHalfBytes, &p.tm_q, &bars.q_full, half * 64,
+                      un.t[t].h, un.t[t].qt * kBM, un.t[t].b);
+      const int b = un.t[0].b, h = un.t[0].h;
+      int kg = 0, vg = 0;    // K / V tiles issued
       bool ok = true;
-      for (int k = 0; ok && k < n_units; ++k, ++uq) {
-        const Unit un = unit_of(p, sched, blockIdx.x, k);
-        const int ns = un.shared ? 1 : 2;   // K/V streams
-        if (uq > 0 && !mbar_wait_bounded(&bars.q_empty, (uq - 1) & 1, abort_flag, p.err,
-                                         kDevErrTimeoutBase | 1u, lim)) {
-          ok = false;
-          break;
+      for (int j = un.j0; ok && j < un.j1; ++j) {
+        {
+          const int st = kg % kKStages, use = kg / kKStages;
+          if (use > 0 && !mbar_wait_bounded(&bars.k_empty[st], (use - 1) & 1, abort_flag, p.err,
+                                            kDevErrTimeoutBase | 2u, lim)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bars.k_full[st], kTileBytes);
+          for (int i = 0; i < 4; ++i) {
+            const SubBox sb = decode_subbox(p, b, 4 * j + i);
+            for (int half = 0; half < 2; ++half)
+              tma_load_4d(smem + kOffK + st * kTileBytes + half * kHalfBytes + i * kSubBytes, &p.tm_k[sb.part],
+                          &bars.k_full[st], half * 64, h, sb.row0, sb.seg);
+          }
+          ++kg;
         }
-        mbar_arrive_expect_tx(&bars.q_full, un.nq * kTileBytes);
-        for (int t = 0; t < un.nq; ++t)
-          for (int half = 0; half < 2; ++half)
-            tma_load_4d(smem + kOffQ + t * kTileBytes + half * kHalfBytes, &p.tm_q, &bars.q_full, half * 64,
-                        un.t[t].h, un.t[t].qt * kBM, un.t[t].b);
-        for (int j = 0; ok && j < T; ++j) {
-          for (int sidx = 0; sidx < ns; ++sidx) {
-            const int st = kg % kKStages, use = kg / kKStages;
-            if (use > 0 && !mbar_wait_bounded(&bars.k_empty[st], (use - 1) & 1, abort_flag, p.err,
-                                              kDevErrTimeoutBase | 2u, lim)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(&bars.k_full[st], kTileBytes);
-            for (int i = 0; i < 4; ++i) {
-              const SubBox sb = decode_subbox(p, un.t[sidx].b, 4 * j + i);
-              for (int half = 0; half < 2; ++half)
-                tma_load_4d(smem + kOffK + st * kTileBytes + half * kHalfBytes + i * kSubBytes,
-                            &p.tm_k[sb.part], &bars.k_full[st], half * 64, un.t[sidx].h, sb.row0, sb.seg);
-            }
-            ++kg;
+        {
+          const int st = vg % kVStages, use = vg / kVStages;
+          if (use > 0 && !mbar_wait_bounded(&bars.v_empty[st], (use - 1) & 1, abort_flag, p.err,
+                                            kDevErrTimeoutBase | 3u, lim)) {
+            ok = false;
+            break;
           }
-          for (int sidx = 0; ok && sidx < ns; ++sidx) {
-            const int st = vg % kVStages, use = vg / kVStages;
-            if (use > 0 && !mbar_wait_bounded(&bars.v_empty[st], (use - 1) & 1, abort_flag, p.err,
-                                              kDevErrTimeoutBase | 3u, lim)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(&bars.v_full[st], kTileBytes);
-            for (int i = 0; i < 4; ++i) {
-              const SubBox sb = decode_subbox(p, un.t[sidx].b, 4 * j + i);
-              for (int half = 0; half < 2; ++half)
-                tma_load_4d(smem + kOffV + st * kTileBytes + half * kHalfBytes + i * kSubBytes,
-                            &p.tm_v[sb.part], &bars.v_full[st], half * 64, un.t[sidx].h, sb.row0, sb.seg);
-            }
-            ++vg;
+          mbar_arrive_expect_tx(&bars.v_full[st], kTileBytes);
+          for (int i = 0; i < 4; ++i) {
+            const SubBox sb = decode_subbox(p, b, 4 * j + i);
+            for (int half = 0; half < 2; ++half)
+              tma_load_4d(smem + kOffV + st * kTileBytes + half * kHalfBytes + i * kSubBytes, &p.tm_v[sb.part],
+                          &bars.v_full[st], half * 64, h, sb.row0, sb.seg);
           }
+          ++vg;
         }
       }
       if (!ok || *abort_flag) {
         // let every load already issued land before the CTA can exit
         const long long short_lim = lim / 4 + 1;
-        if (uq > 0) mbar_wait_bounded(&bars.q_full, (uq - 1) & 1, nullptr, nullptr, 0, short_lim);
+        mbar_wait_bounded(&bars.q_full, 0, nullptr, nullptr, 0, short_lim);
         for (int g = kg - 1; g >= 0 && g >= kg - kKStages; --g)
           mbar_wait_bounded(&bars.k_full[g % kKStages], (g / kKStages) & 1, nullptr, nullptr, 0, short_lim);
         for (int g = vg - 1; g >= 0 && g >= vg - kVStages; --g)
           mbar_wait_bounded(&bars.v_full[g % kVStages], (g / kVStages) & 1, nullptr, nullptr, 0, short_lim);
       }
-    } else if (warp == 1 && lane == 0) {
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       const uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, 0);
       const uint32_t idesc_pv = idesc_bf16_f32(kBM, kHeadDim, 1);
@@ -407,88 +367,61 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
           mma_ts(tO[t], tS[t] + kk * 8, sdesc_sw128(va + kk * 2048, kHalfBytes, 1024), idesc_pv,
                  (!first || kk > 0) ? 1u : 0u);
       };
-      int kg = 0, vg = 0;       // K / V tiles consumed
-      int pc[2] = {0, 0};       // P tiles consumed per query-tile slot
-      int uses[2] = {0, 0};     // units that used each slot
-      int drains = 0, uq = 0;
-      bool ok = true;
       auto wait_k = [&](int g, unsigned site) {
         return mbar_wait_bounded(&bars.k_full[g % kKStages], (g / kKStages) & 1, abort_flag, p.err,
                                  kDevErrTimeoutBase | site, lim);
       };
-      auto drain = [&](unsigned site) {
-        mma_commit(&bars.drain);
-        const bool r = mbar_wait_bounded(&bars.drain, drains & 1, abort_flag, p.err, kDevErrTimeoutBase | site, lim);
-        ++drains;
-        return r;
-      };
-      for (int k = 0; ok && k < n_units; ++k, ++uq) {
-        const Unit un = unit_of(p, sched, blockIdx.x, k);
-        const int nq = un.nq;
-        const int ns = un.shared ? 1 : 2;
-        ok = mbar_wait_bounded(&bars.q_full, uq & 1, abort_flag, p.err, kDevErrTimeoutBase | 4u, lim);
-        if (ok && kDrainBeforeOverwrite && uq > 0) ok = drain(13u);   // last P_t V may still read P_t
-        for (int t = 0; ok && t < nq; ++t) {
-          const int g = kg + (un.shared ? 0 : t);
-          if (t == 0 || !un.shared) ok = wait_k(g, 5u);
-          if (!ok) break;
-          tc_fence_after();
-          issue_qk(t, g % kKStages);
+      int kg = 0, vg = 0, drains = 0;
+      bool ok = mbar_wait_bounded(&bars.q_full, 0, abort_flag, p.err, kDevErrTimeoutBase | 4u, lim);
+      if (ok) ok = wait_k(kg, 5u);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < nq; ++t) {
+          issue_qk(t, kg % kKStages);
           mma_commit(&bars.s_full[t]);
         }
-        if (!ok) break;
-        for (int sidx = 0; sidx < ns; ++sidx) mma_commit(&bars.k_empty[(kg + sidx) % kKStages]);
-        kg += ns;
-        if (T == 1) mma_commit(&bars.q_empty);
-        for (int j = 0; ok && j < T; ++j) {
-          const bool more = j + 1 < T;
-          for (int t = 0; ok && t < nq; ++t) {
-            const int vgt = vg + (un.shared ? 0 : t);
-            if (t == 0 || !un.shared)
-              ok = mbar_wait_bounded(&bars.v_full[vgt % kVStages], (vgt / kVStages) & 1, abort_flag, p.err,
-                                     kDevErrTimeoutBase | 6u, lim);
-            if (ok) ok = mbar_wait_bounded(&bars.p_full[t], pc[t] & 1, abort_flag, p.err, kDevErrTimeoutBase | 7u, lim);
-            if (ok && j == 0 && uses[t] > 0)
-              ok = mbar_wait_bounded(&bars.o_free[t], (uses[t] - 1) & 1, abort_flag, p.err,
-                                     kDevErrTimeoutBase | 8u, lim);
-            if (!ok) break;
-            ++pc[t];
-            tc_fence_after();
-            issue_pv(t, vgt % kVStages, j == 0);
-            if (more) {
-              // S_t of the next tile overwrites P_t
-              if (kDrainBeforeOverwrite) ok = drain(9u);
-              const int g = kg + (un.shared ? 0 : t);
-              if (ok && (t == 0 || !un.shared)) ok = wait_k(g, 10u);
-              if (!ok) break;
-              tc_fence_after();
-              issue_qk(t, g % kKStages);
-              mma_commit(&bars.s_full[t]);
-            }
-          }
+        mma_commit(&bars.k_empty[kg % kKStages]);
+        ++kg;
+      }
+      for (int j = un.j0; ok && j < un.j1; ++j) {
+        const bool more = j + 1 < un.j1;
+        const int vs = vg % kVStages;
+        ok = mbar_wait_bounded(&bars.v_full[vs], (vg / kVStages) & 1, abort_flag, p.err, kDevErrTimeoutBase | 6u,
+                               lim);
+        for (int t = 0; ok && t < nq; ++t) {
+          ok = mbar_wait_bounded(&bars.p_full[t], (j - un.j0) & 1, abort_flag, p.err, kDevErrTimeoutBase | 7u, lim);
           if (!ok) break;
-          for (int sidx = 0; sidx < ns; ++sidx) mma_commit(&bars.v_empty[(vg + sidx) % kVStages]);
-          vg += ns;
+          tc_fence_after();
+          issue_pv(t, vs, j == un.j0);
           if (more) {
-            for (int sidx = 0; sidx < ns; ++sidx) mma_commit(&bars.k_empty[(kg + sidx) % kKStages]);
-            kg += ns;
-            if (j + 1 == T - 1) mma_commit(&bars.q_empty);
+            // S_t of the next tile overwrites P_t
+            if (kDrainBeforeOverwrite) {
+              mma_commit(&bars.drain);
+              ok = mbar_wait_bounded(&bars.drain, drains & 1, abort_flag, p.err, kDevErrTimeoutBase | 9u, lim);
+              ++drains;
+            }
+            if (ok && t == 0) ok = wait_k(kg, 10u);
+            if (!ok) break;
+            tc_fence_after();
+            issue_qk(t, kg % kKStages);
+            mma_commit(&bars.s_full[t]);
           }
         }
         if (!ok) break;
-        for (int t = 0; t < nq; ++t) {
-          mma_commit(&bars.o_final[t]);
-          ++uses[t];
+        mma_commit(&bars.v_empty[vs]);
+        ++vg;
+        if (more) {
+          mma_commit(&bars.k_empty[kg % kKStages]);
+          ++kg;
         }
       }
+      for (int t = 0; t < nq; ++t) mma_commit(&bars.o_final[t]);
       if (!ok) {
         // make sure nothing issued is still running before the memory goes away
-        mma_commit(&bars.drain);
-        mbar_wait_bounded(&bars.drain, drains & 1, nullptr, nullptr, 0, lim / 4 + 1);
+        mbar_wait_bounded(&bars.o_final[0], 0, nullptr, nullptr, 0, lim / 4 + 1);
       }
     }
-  } else {
-    setmaxnreg_inc();
+  } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
     const int t = (warp - 4) >> 2;                 // query-tile slot
     const int quarter = warp & 3;                  // TMEM lane quarter
@@ -497,98 +430,134 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
     const uint32_t tS = tmem + lane_off + t * 128u;
     const uint32_t tO = tmem + lane_off + 256u + t * 128u;
     const float sl2 = p.scale_log2;
-    int sc = 0, oc = 0;                            // S tiles / units consumed
-    bool ok = true;
-    for (int k = 0; ok && k < n_units; ++k) {
-      const Unit un = unit_of(p, sched, blockIdx.x, k);
-      if (t >= un.nq) continue;
-      const QTile qt = un.t[t];
-      float m = -INFINITY;   // running max of scaled scores, base-2 units
-      float l = 0.f;         // running sum of exp2(score - m)
-      for (int j = 0; j < T; ++j) {
-        ok = mbar_wait_bounded(&bars.s_full[t], sc & 1, abort_flag, p.err, kDevErrTimeoutBase | 11u, lim);
-        if (!ok) break;
-        ++sc;
-        tc_fence_after();
-        // which columns hold real keys (most tiles: all of them)
-        const int s0 = 4 * j;
-        int valid[4] = {kSub, kSub, kSub, kSub};
-        const bool check = !p.exact || (s0 + 4 > p.sb_mid_lo && s0 < p.sb_mid_hi) || (s0 + 4 > p.n_sub);
-        if (check) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) valid[i] = subbox_valid(p, s0 + i);
-        }
-        const bool masked = check && (valid[0] != kSub || valid[1] != kSub || valid[2] != kSub || valid[3] != kSub);
-        // the whole row of S in registers: one tensor-memory round trip
-        uint32_t sv[128];
-        tmem_ld128_wait(tS, sv);
-        if (masked) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) mask32(sv + 32 * i, valid[i]);
-        }
-        const float mt = fmaxf(max64(sv), max64(sv + 64)) * sl2;
-        float alpha = 1.f;
-        bool rescale_o = false;
-        if (mt > m + kRescaleThreshold) {
-          alpha = ex2_approx(m - mt);   // 0 when m = -inf
-          l *= alpha;
-          rescale_o = j > 0;
-          m = mt;
-        }
-        const float mb = (m == -INFINITY) ? 0.f : m;
-        const uint64_t sl2x2 = f2_pack(sl2, sl2), nmbx2 = f2_pack(-mb, -mb);
-        uint64_t rs2[2] = {0ull, 0ull};
-        // P = exp2(S * scale - m) as bf16 pairs, written over S
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) exp_chunk(sv + 32 * cc, tS + cc * 16, sl2x2, nmbx2, rs2);
-        {
-          const uint64_t r = f2_add(rs2[0], rs2[1]);
-          l += f2_lo(r) + f2_hi(r);
-        }
-        if (rescale_o) {
-          // O holds every P V up to the previous tile (completed before S of
-          // this tile was signalled); the next P V is issued after p_full
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            uint32_t o[32];
-            tmem_ld32_wait(tO + cc * 32, o);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tO + cc * 32, o);
-          }
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&bars.p_full[t]);
-      }
-      if (ok) ok = mbar_wait_bounded(&bars.o_final[t], oc & 1, abort_flag, p.err, kDevErrTimeoutBase | 12u, lim);
+    bool ok = t < nq;
+    float m = -INFINITY;   // running max of scaled scores, base-2 units
+    float l = 0.f;         // running sum of exp2(score - m)
+    for (int j = un.j0; ok && j < un.j1; ++j) {
+      ok = mbar_wait_bounded(&bars.s_full[t], (j - un.j0) & 1, abort_flag, p.err, kDevErrTimeoutBase | 11u, lim);
       if (!ok) break;
-      ++oc;
       tc_fence_after();
+      // which columns hold real keys (most tiles: all of them)
+      const int s0 = 4 * j;
+      int valid[4] = {kSub, kSub, kSub, kSub};
+      const bool check = !p.exact || (s0 + 4 > p.sb_mid_lo && s0 < p.sb_mid_hi) || (s0 + 4 > p.n_sub);
+      if (check) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) valid[i] = subbox_valid(p, s0 + i);
+      }
+      const bool masked = check && (valid[0] != kSub || valid[1] != kSub || valid[2] != kSub || valid[3] != kSub);
+      // the whole row of S in registers: one tensor-memory round trip
+      uint32_t sv[128];
+      tmem_ld128_wait(tS, sv);
+      if (masked) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mask32(sv + 32 * i, valid[i]);
+      }
+      const float mt = fmaxf(max64(sv), max64(sv + 64)) * sl2;
+      float alpha = 1.f;
+      bool rescale_o = false;
+      if (mt > m + kRescaleThreshold) {
+        alpha = ex2_approx(m - mt);   // 0 when m = -inf
+        l *= alpha;
+        rescale_o = j > un.j0;
+        m = mt;
+      }
+      const float mb = (m == -INFINITY) ? 0.f : m;
+      const uint64_t sl2x2 = f2_pack(sl2, sl2), nmbx2 = f2_pack(-mb, -mb);
+      uint64_t rs2[2] = {0ull, 0ull};
+      // P = exp2(S * scale - m) as bf16 pairs, written over S
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) exp_chunk(sv + 32 * cc, tS + cc * 16, sl2x2, nmbx2, rs2);
+      {
+        const uint64_t r = f2_add(rs2[0], rs2[1]);
+        l += f2_lo(r) + f2_hi(r);
+      }
+      if (rescale_o) {
+        // O holds every P V up to the previous tile (completed before S of
+        // this tile was signalled); the next P V is issued after p_full
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          tmem_ld32_wait(tO + cc * 32, o);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tO + cc * 32, o);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars.p_full[t]);
+    }
+    if (ok) ok = mbar_wait_bounded(&bars.o_final[t], 0, abort_flag, p.err, kDevErrTimeoutBase | 12u, lim);
+    if (ok) {
+      tc_fence_after();
+      const QTile qt = un.t[t];
       const int qrow = qt.qt * kBM + row;
-      const float inv = 1.f / l;
       __nv_bfloat16* O = static_cast<__nv_bfloat16*>(p.O);
       uint4* dst = reinterpret_cast<uint4*>(O + ((static_cast<long long>(qt.b) * p.n + qrow) * p.H + qt.h) * kHeadDim);
+      if (un.tail < 0) {
+        const float inv = 1.f / l;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t o[32];
-        tmem_ld32_wait(tO + cc * 32, o);
-        if (qrow < p.n) {
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          tmem_ld32_wait(tO + cc * 32, o);
+          if (qrow < p.n) store_row_bf16(dst + cc * 4, reinterpret_cast<const float*>(o), inv);
+        }
+        if (p.lse != nullptr && qrow < p.n)
+          p.lse[(static_cast<long long>(qt.b) * p.H + qt.h) * p.n + qrow] = (m + __log2f(l)) * 0.69314718055994531f;
+      } else {
+        // tail chunk: park the unnormalised row, then the last chunk merges
+        const int K = p.tail_chunks;
+        const long long slot = static_cast<long long>(un.tail) * K + un.chunk;
+        float4* po = reinterpret_cast<float4*>(p.part_o + (slot * kBM + row) * kHeadDim);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
-            dst[cc * 4 + v] = w;
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          tmem_ld32_wait(tO + cc * 32, o);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            po[cc * 8 + v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                         __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+        }
+        p.part_ml[(slot * 2 + 0) * kBM + row] = m;
+        p.part_ml[(slot * 2 + 1) * kBM + row] = l;
+        __threadfence();
+        named_sync(1, kBM);
+        if (row == 0) bars.merge = (atomicAdd(&p.tail_ticket[un.tail], 1u) == static_cast<unsigned>(K - 1)) ? 1 : 0;
+        named_sync(1, kBM);
+        if (bars.merge) {
+          __threadfence();
+          const long long base = static_cast<long long>(un.tail) * K;
+          float M = -INFINITY;
+          for (int c = 0; c < K; ++c) M = fmaxf(M, __ldcg(p.part_ml + ((base + c) * 2) * kBM + row));
+          float L = 0.f;
+          float acc[kHeadDim];
+#pragma unroll
+          for (int d = 0; d < kHeadDim; ++d) acc[d] = 0.f;
+          for (int c = 0; c < K; ++c) {
+            const float mc = __ldcg(p.part_ml + ((base + c) * 2) * kBM + row);
+            const float w = ex2_approx(mc - M);
+            L += w * __ldcg(p.part_ml + ((base + c) * 2 + 1) * kBM + row);
+            const float4* src = reinterpret_cast<const float4*>(p.part_o + ((base + c) * kBM + row) * kHeadDim);
+#pragma unroll
+            for (int v = 0; v < kHeadDim / 4; ++v) {
+              const float4 x = __ldcg(src + v);
+              acc[4 * v + 0] = fmaf(w, x.x, acc[4 * v + 0]);
+              acc[4 * v + 1] = fmaf(w, x.y, acc[4 * v + 1]);
+              acc[4 * v + 2] = fmaf(w, x.z, acc[4 * v + 2]);
+              acc[4 * v + 3] = fmaf(w, x.w, acc[4 * v + 3]);
+            }
           }
+          if (qrow < p.n) {
+            const float inv = 1.f / L;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) store_row_bf16(dst + cc * 4, acc + 32 * cc, inv);
+            if (p.lse != nullptr)
+              p.lse[(static_cast<long long>(qt.b) * p.H + qt.h) * p.n + qrow] = (M + __log2f(L)) * 0.69314718055994531f;
+          }
+          if (row == 0) p.tail_ticket[un.tail] = 0u;   // ready for the next launch
         }
       }
-      tc_fence_before();
-      mbar_arrive(&bars.o_free[t]);
-      if (p.lse != nullptr && qrow < p.n)
-        p.lse[(static_cast<long long>(qt.b) * p.H + qt.h) * p.n + qrow] = (m + __log2f(l)) * 0.69314718055994531f;
     }
   }
 
@@ -617,21 +586,26 @@ __global__ void wait_timeout_kernel(unsigned* err, long long lim) {
 
 }  // namespace
 
+int attend_tail_chunks(int B, int H, int q_tiles, int n_tiles) {
+  if ((q_tiles & 1) == 0) return 1;
+  const int tails = B * H;
+  int k = kAttendMaxTailSlots / tails;
+  if (k > kAttendMaxChunksPerTail) k = kAttendMaxChunksPerTail;
+  if (k > n_tiles) k = n_tiles;
+  return k < 1 ? 1 : k;
+}
+
 cudaError_t launch_attend(const AttendParams& p, cudaStream_t st) {
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
+    attr_set = true;
   }
-  const int bh = p.B * p.H;
-  const int units = bh * (p.q_tiles / 2) + ((p.q_tiles & 1) ? bh : 0);
-  const int grid = PF_ATTEND_ONE_UNIT_PER_CTA ? units : (units < sms ? units : sms);
-  attend_kernel<<<grid, kThreads, kSmemBytes, st>>>(p);
+  const long long bh = 1LL * p.B * p.H;
+  const long long units = bh * (p.q_tiles / 2) + ((p.q_tiles & 1) ? bh * p.tail_chunks : 0);
+  if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
+  attend_kernel<<<static_cast<unsigned>(units), kThreads, kSmemBytes, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -47,6 +47,10 @@ constexpr int kMaxPoolSlots = 8192;                         // the top-k keeps a
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
+// attention scratch shared by all layers: split-tail partial outputs, row
+// statistics and tickets
+constexpr size_t kAttendScratchBytes = pf::kAttendPartOBytes + pf::kAttendPartMLBytes + pf::kAttendTicketBytes;
+
 struct Geometry {
   int n, n_c, slots, HD;
   size_t sink_bytes, pool_bytes, recent_bytes;  // per K (or V) tensor
@@ -154,6 +158,9 @@ struct pf_cache {
   char* arena;
   size_t arena_bytes;
   unsigned* err;  // device error word
+  float* part_o;
+  float* part_ml;
+  unsigned* tail_ticket;
   long long timeout_cycles;
   std::vector<Layer> L;
 };
@@ -266,7 +273,7 @@ pf_status pf_cache_bytes(const pf_config* cfg, size_t* bytes) {
   if (s != PF_OK) return s;
   if (bytes == nullptr) return fail(PF_ERR_ARG, "bytes is NULL");
   const Geometry g = geometry(cfg);
-  *bytes = kAlign /* error word */ + g.layer_bytes * static_cast<size_t>(cfg->layers);
+  *bytes = kAlign /* error word */ + kAttendScratchBytes + g.layer_bytes * static_cast<size_t>(cfg->layers);
   return PF_OK;
 }
 
@@ -288,6 +295,9 @@ pf_status pf_cache_create(const pf_config* cfg, void* dev_arena, size_t arena_by
   c->timeout_cycles = kDefaultTimeoutCycles;
   c->L.resize(cfg->layers);
   char* p = c->arena + kAlign;
+  c->part_o = reinterpret_cast<float*>(p); p += pf::kAttendPartOBytes;
+  c->part_ml = reinterpret_cast<float*>(p); p += pf::kAttendPartMLBytes;
+  c->tail_ticket = reinterpret_cast<unsigned*>(p); p += pf::kAttendTicketBytes;
   for (int l = 0; l < cfg->layers; ++l) {
     Layer& Ly = c->L[l];
     const Geometry& g = c->g;
@@ -636,6 +646,10 @@ pf_status pf_attend(pf_cache* c, int layer, const void* Q, const void* K_cur, co
   p.sb_mid_hi = p.sb_sink + n_sel * p.sb_mid;
   p.exact = (sink_rows % 32 == 0 && g.n % 32 == 0) ? 1 : 0;
   p.q_tiles = (g.n + 127) / 128;
+  p.tail_chunks = pf::attend_tail_chunks(B, H, p.q_tiles, p.n_tiles);
+  p.part_o = c->part_o;
+  p.part_ml = c->part_ml;
+  p.tail_ticket = c->tail_ticket;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
   p.err = c->err;
   p.timeout_cycles = c->timeout_cycles;

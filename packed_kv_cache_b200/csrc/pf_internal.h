@@ -87,10 +87,23 @@ struct AttendParams {
   int exact;            // sink rows and block rows are multiples of 32: only mid blocks and
                         // the padding after the last key have partial sub-boxes
   int q_tiles;          // 128-row query tiles per (b, h)
+  int tail_chunks;      // context chunks each ragged last query tile is split into (1 = not split)
+  float* part_o;        // [tails * tail_chunks, 128, 128] unnormalised partial outputs
+  float* part_ml;       // [tails * tail_chunks, 2, 128] partial row max / row sum
+  unsigned* tail_ticket;  // [tails], zero on entry, left zero on exit
   float scale_log2;     // log2(e) / sqrt(D)
   unsigned* err;
   long long timeout_cycles;
 };
+
+// Scratch for split tails, in the cache arena: kAttendMaxTailSlots chunk
+// slots of partial outputs and row statistics, and one ticket per tail.
+constexpr int kAttendMaxTailSlots = 256;
+constexpr int kAttendMaxChunksPerTail = 8;
+constexpr size_t kAttendPartOBytes = size_t(kAttendMaxTailSlots) * 128 * 128 * 4;
+constexpr size_t kAttendPartMLBytes = size_t(kAttendMaxTailSlots) * 2 * 128 * 4;
+constexpr size_t kAttendTicketBytes = size_t(kAttendMaxTailSlots) * 4;
+int attend_tail_chunks(int B, int H, int q_tiles, int n_tiles);
 
 cudaError_t launch_attend(const AttendParams& p, cudaStream_t st);
 

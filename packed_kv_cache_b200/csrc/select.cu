@@ -111,7 +111,7 @@ __device__ unsigned block_exclusive_scan(unsigned v, unsigned* total) {
   return before + x - v;
 }
 
-__global__ void __launch_bounds__(kThreads) score_kernel(const SelectArgs a) {
+__global__ void __launch_bounds__(kThreads, 5) score_kernel(const SelectArgs a) {
   extern __shared__ float smem[];
   float* qs = smem;                                      // [HD]
   uint32_t* keys = reinterpret_cast<uint32_t*>(smem + a.HD);  // [count]
@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(kThreads) score_kernel(const SelectArgs a) {
                    ((static_cast<long long>(b) * a.slots + slot) * a.n_c + row_lo) * G;
   const int nu = rows * G;
   float acc = 0.f;
-  constexpr int U = 8;
+  constexpr int U = 6;
   for (int u0 = t; u0 < nu; u0 += kThreads * U) {
     uint4 w[U];
 #pragma unroll
@@ -194,16 +194,16 @@ __global__ void __launch_bounds__(kThreads) score_kernel(const SelectArgs a) {
         if (shift == 24 || (key >> (shift + 8)) == (pre >> (shift + 8))) atomicAdd(&hist[(key >> shift) & 255u], 1u);
       }
       __syncthreads();
-      if (t == 0) {
-        unsigned cum = 0u;
-        for (int d = 255; d >= 0; --d) {
-          const unsigned hc = hist[d];
-          if (cum + hc >= sh_need) {
-            sh_prefix = pre | (static_cast<unsigned>(d) << shift);
-            sh_need -= cum;
-            break;
-          }
-          cum += hc;
+      {
+        // suffix sums over the digits, from 255 down: thread t holds digit 255 - t
+        const unsigned hc = hist[255 - t];
+        unsigned tot;
+        const unsigned before = block_exclusive_scan(hc, &tot);   // count of digits > 255 - t
+        const unsigned need = sh_need;
+        __syncthreads();
+        if (before < need && before + hc >= need) {               // exactly one thread
+          sh_prefix = pre | (static_cast<unsigned>(255 - t) << shift);
+          sh_need = need - before;
         }
       }
       __syncthreads();

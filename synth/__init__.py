@@ -15,8 +15,9 @@ dims; "Implementation Details" and Sec. 3.2 "Compressed Mid Tokens"):
 * ``step30``    the same per-layer shapes with a 116-block pool, 30 layers.
 * ``dense``     a 748,800-key full-resolution context, no mid pool.
 * ``stress16`` / ``stress64``  batch 2, a 1,000-block pool, top-16 / top-64.
-* ``ragged_a`` / ``ragged_b``  small test shapes whose block and pool sizes are
-  not multiples of any tile size, to exercise ragged tails.
+* ``ragged_a`` / ``ragged_b`` / ``ragged_c``  small test shapes whose block
+  and pool sizes are not multiples of any tile size, to exercise ragged tails
+  (``ragged_c`` has an odd number of 128-row query tiles).
 
 Values are N(0,1) drawn by torch's generators and rounded to bf16.  Planted
 mid blocks follow the recipe K~ = 0.8 * mean_i(Q_i) + 0.2 * N(0,1), with the
@@ -71,6 +72,8 @@ WORKLOADS = {
     # multiples of 32, the pool is not a multiple of anything.
     "ragged_a": Workload("ragged_a", 2, 2, 128, 4, 6, 10, 240, 4, 2, 1, 13, 13, 5, 5, 1, 32),
     "ragged_b": Workload("ragged_b", 1, 3, 128, 2, 9, 13, 234, 6, 1, 2, 11, 16, 4, 4, 1, 32),
+    # an odd number (3) of 128-row query tiles: the last tile is split along the context
+    "ragged_c": Workload("ragged_c", 2, 3, 128, 4, 6, 14, 336, 6, 2, 1, 9, 9, 4, 4, 1, 32),
 }
 
 SEED_BASE = 1000

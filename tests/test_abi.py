@@ -62,10 +62,13 @@ def test_cache_bytes_layout(pf):
     cpb = (182 + 31) // 32
     per_layer = (2 * (al(2 * 6240 * row) + al(slots * 182 * row) + al(6240 * row))
                  + al(16 * 4) + al(slots * 4) + al(slots * cpb * 4) + al(12 * 128 * 4) + al(4))
-    assert got == 256 + per_layer
+    # shared attention scratch: 256 split-tail slots of 128x128 fp32 partial
+    # outputs, their row max / row sum, and 256 tickets
+    scratch = 256 * 128 * 128 * 4 + 256 * 2 * 128 * 4 + 256 * 4
+    assert got == 256 + scratch + per_layer
     # layers scale linearly
     c.layers = 30
-    assert pf.pf_cache_bytes(c) == 256 + 30 * per_layer
+    assert pf.pf_cache_bytes(c) == 256 + scratch + 30 * per_layer
 
 
 @pytest.mark.parametrize("field,value,status", [

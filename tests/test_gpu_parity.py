@@ -114,7 +114,8 @@ def test_rope_shift_stress_full_size(pf):
 
 # ------------------------------------------------------------------ selection
 
-@pytest.mark.parametrize("name", ["tiny", "ragged_a", "ragged_b", "layer", "step30", "stress16", "stress64"])
+@pytest.mark.parametrize("name", ["tiny", "ragged_a", "ragged_b", "ragged_c", "layer", "step30", "stress16",
+                                  "stress64"])
 def test_selection_bit_exact(pf, name):
     wl = _wl(name)
     d = synth.make_layer(wl, seed_for(name), device="cpu", with_values=False)
@@ -192,10 +193,23 @@ def _attend_and_compare(pf, wl, d, rows=None, via_append=False, lse_check=True):
     return res
 
 
-@pytest.mark.parametrize("name", ["tiny", "ragged_a", "ragged_b"])
+@pytest.mark.parametrize("name", ["tiny", "ragged_a", "ragged_b", "ragged_c"])
 def test_attention_small_full(pf, name):
     wl, d = _layer(name)
     _attend_and_compare(pf, wl, d)
+
+
+def test_attention_split_tail_repeated_calls(pf):
+    # the split-tail scratch (partial outputs, tickets) is reused across calls
+    wl, d = _layer("ragged_c")
+    cache = build_cache(pf, wl, d)
+    Q, Kc, Vc = d["Q"].cuda(), d["K_cur"].cuda(), d["V_cur"].cuda()
+    s = torch.zeros((wl.batch, wl.n_top), dtype=torch.int32, device="cuda")
+    cache.select_mid(0, Q, s, None)
+    outs = [cache.attend(0, Q, Kc, Vc).cpu() for _ in range(3)]
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
+    O_ref, _ = oracle.attend(d["Q"], oracle_context(wl, d, s.cpu().numpy()))
+    assert_attention_close(outs[2], O_ref, "ragged_c repeated")
 
 
 def test_attention_pool_filled_by_appends(pf):
