@@ -481,7 +481,9 @@ def run_suite(args):
             row = H * D * 2
             if name == "stress16":
                 ms = _timed(lambda: cache.select_mid(0, d["Q"]), iters, flush, stream)
-                out.append(line("select (qpool + score + top-k)", name, ms, "hbm", B * (n + P * nc) * row, None))
+                # reads: the queries (bf16) and each block's cached mean key (fp32)
+                out.append(line("select (qpool + mean-key scores + top-k)", name, ms, "hbm",
+                                B * n * row + B * P * H * D * 4, None))
                 parts = pf.PART_SINK | pf.PART_MID | pf.PART_RECENT
                 ms = _timed(lambda: cache.rope_shift(0, parts, 4), iters, flush, stream)
                 rows = B * (wl.sink_blocks * n + P * nc + wl.recent_blocks * (n + nc))

@@ -63,6 +63,12 @@ constexpr float kRescaleThreshold = 8.0f;
 #define PF_ATTEND_DRAIN 0
 #endif
 constexpr bool kDrainBeforeOverwrite = PF_ATTEND_DRAIN != 0;
+// The MMA issuer polls both query tiles' P barriers and serves the first
+// ready (1; measured slower: the spinning thread takes issue slots from the
+// softmax warps), or waits for tile 0 then tile 1 (0).
+#ifndef PF_ATTEND_MMA_POLL
+#define PF_ATTEND_MMA_POLL 0
+#endif
 // One exponential pair in kPolyPeriod is evaluated by ex2_poly (FMA pipe),
 // the others by the special-function unit (0 = never; measured slower).
 #ifndef PF_ATTEND_POLY_PERIOD
@@ -388,6 +394,42 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
         const int vs = vg % kVStages;
         ok = mbar_wait_bounded(&bars.v_full[vs], (vg / kVStages) & 1, abort_flag, p.err, kDevErrTimeoutBase | 6u,
                                lim);
+#if PF_ATTEND_MMA_POLL
+        // serve the two query tiles in whichever order their P becomes ready
+        {
+          const uint32_t ph = (j - un.j0) & 1;
+          bool served[2] = {false, nq < 2};
+          bool k_ready = !more;
+          const long long t0 = clock64();
+          while (ok && !(served[0] && served[1])) {
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              if (served[t] || !mbar_test_wait(&bars.p_full[t], ph)) continue;
+              tc_fence_after();
+              issue_pv(t, vs, j == un.j0);
+              if (more) {
+                if (!k_ready) {
+                  ok = wait_k(kg, 10u);
+                  k_ready = ok;
+                  if (!ok) break;
+                  tc_fence_after();
+                }
+                issue_qk(t, kg % kKStages);   // S_t of the next tile overwrites P_t
+                mma_commit(&bars.s_full[t]);
+              }
+              served[t] = true;
+            }
+            if (ok && !(served[0] && served[1])) {
+              if (*abort_flag) ok = false;
+              else if (clock64() - t0 > lim) {
+                *abort_flag = 1;
+                atomicCAS(p.err, 0u, kDevErrTimeoutBase | 7u);
+                ok = false;
+              }
+            }
+          }
+        }
+#else
         for (int t = 0; ok && t < nq; ++t) {
           ok = mbar_wait_bounded(&bars.p_full[t], (j - un.j0) & 1, abort_flag, p.err, kDevErrTimeoutBase | 7u, lim);
           if (!ok) break;
@@ -407,6 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
             mma_commit(&bars.s_full[t]);
           }
         }
+#endif
         if (!ok) break;
         mma_commit(&bars.v_empty[vs]);
         ++vg;

@@ -54,7 +54,7 @@ constexpr size_t kAttendScratchBytes = pf::kAttendPartOBytes + pf::kAttendPartML
 struct Geometry {
   int n, n_c, slots, HD;
   size_t sink_bytes, pool_bytes, recent_bytes;  // per K (or V) tensor
-  size_t sel_bytes, scores_bytes, partial_bytes, qsum_bytes, ticket_bytes;
+  size_t sel_bytes, scores_bytes, partial_bytes, qsum_bytes, ticket_bytes, kbar_bytes;
   size_t layer_bytes;
   int chunk_rows, chunks_per_block;
 };
@@ -102,8 +102,9 @@ Geometry geometry(const pf_config* c) {
   g.partial_bytes = align_up(B * g.slots * g.chunks_per_block * 4);
   g.qsum_bytes = align_up(B * g.HD * 4);
   g.ticket_bytes = align_up(B * 4);
+  g.kbar_bytes = align_up(B * g.slots * g.HD * 4);
   g.layer_bytes = 2 * (g.sink_bytes + g.pool_bytes + g.recent_bytes) + g.sel_bytes + g.scores_bytes +
-                  g.partial_bytes + g.qsum_bytes + g.ticket_bytes;
+                  g.partial_bytes + g.qsum_bytes + g.ticket_bytes + g.kbar_bytes;
   return g;
 }
 
@@ -118,6 +119,7 @@ struct Layer {
   int32_t* sel;
   float *scores, *partial, *qsum;
   unsigned* ticket;
+  float* kbar;  // [B, slots, H * D] mean key of each pool slot
 };
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -201,11 +203,12 @@ struct RunBuilder {
   pf::RowRuns runs;
   pf::RopeTable tab;
   cudaStream_t st;
+  bool f32 = false;  // runs of float32 vectors (cached mean keys) instead of bf16 keys
   cudaError_t err = cudaSuccess;
   RunBuilder() { runs.n = 0; runs.start[0] = 0; }
   void flush() {
     if (runs.n == 0) return;
-    cudaError_t e = pf::launch_rope_shift(runs, tab, st);
+    cudaError_t e = f32 ? pf::launch_rope_shift_f32(runs, tab, st) : pf::launch_rope_shift(runs, tab, st);
     if (e != cudaSuccess && err == cudaSuccess) err = e;
     runs.n = 0;
     runs.start[0] = 0;
@@ -312,6 +315,7 @@ pf_status pf_cache_create(const pf_config* cfg, void* dev_arena, size_t arena_by
     Ly.partial = reinterpret_cast<float*>(p); p += g.partial_bytes;
     Ly.qsum = reinterpret_cast<float*>(p); p += g.qsum_bytes;
     Ly.ticket = reinterpret_cast<unsigned*>(p); p += g.ticket_bytes;
+    Ly.kbar = reinterpret_cast<float*>(p); p += g.kbar_bytes;
   }
   cudaError_t e = cudaMemsetAsync(c->arena, 0, need, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
@@ -414,6 +418,12 @@ pf_status pf_cache_append_block(pf_cache* c, int layer, const void* K, const voi
   nx.blocks_seen += 1;
   cb.flush();
   if (cb.err != cudaSuccess) return cuda_fail(cb.err, "append copy launch");
+  if (!to_sink && Kc != nullptr && Vc != nullptr) {
+    const int pslot = (nx.mid_head + nx.mid_count + nx.recent_count - 1) % g.slots;
+    cudaError_t e = pf::launch_kmean(Ly.pool_k, Ly.kbar, cf.batch, g.slots, g.n_c, g.HD, pslot, 1,
+                                     static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "append key-mean launch");
+  }
   Ly = nx;
   if (evicted) *evicted = ev;
   return PF_OK;
@@ -473,6 +483,14 @@ pf_status pf_cache_load_mid(pf_cache* c, int layer, const void* Kc, const void* 
   nx.sel_valid = false;
   cb.flush();
   if (cb.err != cudaSuccess) return cuda_fail(cb.err, "load_mid copy launch");
+  for (int i = 0; i < keep;) {
+    const int slot = (start_slot + i) % g.slots;
+    const int run = (g.slots - slot) < (keep - i) ? (g.slots - slot) : (keep - i);
+    cudaError_t e = pf::launch_kmean(Ly.pool_k, Ly.kbar, cf.batch, g.slots, g.n_c, g.HD, slot, run,
+                                     static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "load_mid key-mean launch");
+    i += run;
+  }
   Ly = nx;
   if (evicted) *evicted = ev;
   return PF_OK;
@@ -497,13 +515,14 @@ pf_status pf_select_mid(pf_cache* c, int layer, const void* Q, int32_t* sel_out,
   a.HD = g.HD;
   a.qsum = Ly.qsum;
   a.pool_k = Ly.pool_k;
+  a.kbar = Ly.kbar;
   a.slots = g.slots;
   a.n_c = g.n_c;
   a.head = Ly.mid_head;
   a.count = Ly.mid_count;
   a.chunk_rows = g.chunk_rows;
-  a.chunks_per_block = g.chunks_per_block;
-  a.score_scale = static_cast<float>(1.0 / (static_cast<double>(g.n) * g.n_c * cf.heads * std::sqrt(128.0)));
+  a.chunks_per_block = 1;   // one partial per block: the dot product with its mean key
+  a.score_scale = static_cast<float>(1.0 / (static_cast<double>(g.n) * cf.heads * std::sqrt(128.0)));
   a.partial = Ly.partial;
   a.scores = Ly.scores;
   a.ticket = Ly.ticket;
@@ -527,8 +546,10 @@ pf_status pf_rope_shift(pf_cache* c, int layer, unsigned parts, int delta, void*
   if (parts & ~(PF_PART_SINK | PF_PART_MID | PF_PART_RECENT)) return fail(PF_ERR_ARG, "unknown partition bits");
   const pf_config& cf = c->cfg;
   const Geometry& g = c->g;
-  RunBuilder rb;
+  RunBuilder rb, rm;
   rb.st = static_cast<cudaStream_t>(stream);
+  rm.st = rb.st;
+  rm.f32 = true;
   rb.tab.pairs = cf.rope_split[0] / 2;
   for (int k = 0; k < 32; ++k) {
     rb.tab.c[k] = 1.f;
@@ -540,6 +561,7 @@ pf_status pf_rope_shift(pf_cache* c, int layer, unsigned parts, int delta, void*
     rb.tab.c[k] = static_cast<float>(std::cos(ang));
     rb.tab.s[k] = static_cast<float>(std::sin(ang));
   }
+  rm.tab = rb.tab;
   if (delta == 0 || parts == 0) return PF_OK;
   const int l0 = layer < 0 ? 0 : layer, l1 = layer < 0 ? cf.layers : layer + 1;
   const long long H = cf.heads;
@@ -571,9 +593,27 @@ pf_status pf_rope_shift(pf_cache* c, int layer, unsigned parts, int delta, void*
       if (cf.mid_capacity > 0)
         add_ring(Ly.pool_k, g.slots, (Ly.mid_head + Ly.mid_count) % g.slots, Ly.recent_count, g.n_c);
     }
+    // the cached mean keys rotate with their blocks (the mean of rotated keys
+    // is the rotated mean)
+    auto add_mean_ring = [&](int head, int count) {
+      for (int b = 0; b < cf.batch; ++b) {
+        int i = 0;
+        while (i < count) {
+          const int slot = (head + i) % g.slots;
+          const int run = (g.slots - slot) < (count - i) ? (g.slots - slot) : (count - i);
+          rm.add(Ly.kbar + (static_cast<size_t>(b) * g.slots + slot) * g.HD, 1LL * run * H);
+          i += run;
+        }
+      }
+    };
+    if (parts & PF_PART_MID) add_mean_ring(Ly.mid_head, Ly.mid_count);
+    if ((parts & PF_PART_RECENT) && cf.mid_capacity > 0)
+      add_mean_ring((Ly.mid_head + Ly.mid_count) % g.slots, Ly.recent_count);
   }
   rb.flush();
+  rm.flush();
   if (rb.err != cudaSuccess) return cuda_fail(rb.err, "rope shift launch");
+  if (rm.err != cudaSuccess) return cuda_fail(rm.err, "rope shift (mean keys) launch");
   if (parts & PF_PART_SINK)
     for (int l = l0; l < l1; ++l) c->L[l].total_shift += delta;
   return PF_OK;

@@ -30,6 +30,8 @@ struct RopeTable {
 };
 
 cudaError_t launch_rope_shift(const RowRuns& runs, const RopeTable& tab, cudaStream_t st);
+// The same rotation of float32 128-dim vectors (cached mean keys); runs count vectors.
+cudaError_t launch_rope_shift_f32(const RowRuns& runs, const RopeTable& tab, cudaStream_t st);
 
 // ------------------------------------------------------------- copies
 // start[] = prefix sums of run lengths in 16-byte units.
@@ -48,6 +50,7 @@ struct SelectArgs {
   int B, n, HD;         // HD = H * D
   float* qsum;          // [B, HD] accumulator, zero on entry, left zero on exit
   const void* pool_k;   // [B, slots, n_c, H, D] bf16
+  const float* kbar;    // [B, slots, HD] mean key per pool slot, or null: stream pool_k
   int slots, n_c;
   int head, count;      // live blocks: age p -> slot (head + p) % slots
   int chunk_rows;       // pool rows per scoring CTA
@@ -63,6 +66,10 @@ struct SelectArgs {
 };
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
+
+// kbar[b, slot] = mean of the block's n_c keys, slots [slot0, slot0 + nslots).
+cudaError_t launch_kmean(const void* pool_k, float* kbar, int B, int slots, int n_c, int HD, int slot0, int nslots,
+                         cudaStream_t st);
 
 // ------------------------------------------------------------- attention
 // Partition ids of the K/V tensor maps.

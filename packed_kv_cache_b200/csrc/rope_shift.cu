@@ -15,6 +15,10 @@
 
 #include "pf_internal.h"
 
+#ifndef PF_ROPE_COOP
+#define PF_ROPE_COOP 0
+#endif
+
 namespace pf {
 
 namespace {
@@ -69,6 +73,60 @@ __global__ void __launch_bounds__(256) rope_shift_kernel(const RowRuns runs, con
   }
 }
 
+// Warp-cooperative form: lane l of a warp owns 16-byte word (l % NW) of key
+// vector (l / NW) of a group of 32 / NW vectors, so one load instruction of
+// the warp reads NW * 16 contiguous bytes per vector; each lane keeps the
+// cosines and sines of its own four pairs in registers.  kGroups groups of
+// vectors are in flight per thread.
+template <int NW>
+__global__ void __launch_bounds__(256) rope_shift_coop_kernel(const RowRuns runs, const RopeTable tab) {
+  constexpr int kPerWarp = 32 / NW;  // vectors per warp step
+  constexpr int kGroups = 4;
+  const int lane = threadIdx.x & 31;
+  const int word = lane % NW, vsub = lane / NW;
+  const bool active = vsub < kPerWarp;
+  float cs[4], sn[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int pair = word * 4 + q;
+    cs[q] = pair < tab.pairs ? tab.c[pair] : 1.f;
+    sn[q] = pair < tab.pairs ? tab.s[pair] : 0.f;
+  }
+  const long long total = runs.start[runs.n];
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
+  const long long wid = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
+  int seg = 0;
+  for (long long base = wid * kPerWarp * kGroups; base < total; base += warps * kPerWarp * kGroups) {
+    uint4 w[kGroups];
+    uint4* ptr[kGroups];
+#pragma unroll
+    for (int g = 0; g < kGroups; ++g) {
+      const long long i = base + g * kPerWarp + vsub;
+      ptr[g] = nullptr;
+      if (active && i < total) {
+        while (i >= runs.start[seg + 1]) ++seg;
+        while (i < runs.start[seg]) --seg;
+        ptr[g] = reinterpret_cast<uint4*>(static_cast<char*>(runs.ptr[seg]) + (i - runs.start[seg]) * (kHeadDim * 2)) + word;
+        w[g] = *ptr[g];
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < kGroups; ++g) {
+      if (ptr[g] != nullptr) {
+        uint32_t v[4] = {w[g].x, w[g].y, w[g].z, w[g].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&v[q]);
+          const float re = __low2float(x), im = __high2float(x);
+          __nv_bfloat162 y = __floats2bfloat162_rn(re * cs[q] - im * sn[q], re * sn[q] + im * cs[q]);
+          v[q] = *reinterpret_cast<uint32_t*>(&y);
+        }
+        *ptr[g] = make_uint4(v[0], v[1], v[2], v[3]);
+      }
+    }
+  }
+}
+
 template <int NW>
 cudaError_t launch_nw(const RowRuns& runs, const RopeTable& tab, cudaStream_t st) {
   static int grid_cap = 0;
@@ -76,17 +134,62 @@ cudaError_t launch_nw(const RowRuns& runs, const RopeTable& tab, cudaStream_t st
     int dev = 0, sms = 148, per_sm = 1;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+#if PF_ROPE_COOP
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rope_shift_coop_kernel<NW>, 256, 0);
+#else
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rope_shift_kernel<NW>, 256, 0);
+#endif
     grid_cap = sms * (per_sm > 0 ? per_sm : 1);
   }
   const long long total = runs.start[runs.n];
+#if PF_ROPE_COOP
+  const long long want = (total + 8 * (32 / NW) * 4 - 1) / (8 * (32 / NW) * 4);
+  const int grid = static_cast<int>(want < grid_cap ? want : grid_cap);
+  rope_shift_coop_kernel<NW><<<grid, 256, 0, st>>>(runs, tab);
+#else
   const long long want = (total + 511) / 512;
   const int grid = static_cast<int>(want < grid_cap ? want : grid_cap);
   rope_shift_kernel<NW><<<grid, 256, 0, st>>>(runs, tab);
+#endif
   return cudaGetLastError();
 }
 
+// float32 vectors: the first ceil(pairs / 2) float4 words of each 128-float vector.
+__global__ void __launch_bounds__(256) rope_shift_f32_kernel(const RowRuns runs, const RopeTable tab) {
+  const long long total = runs.start[runs.n];
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  const int words = (tab.pairs + 1) / 2;
+  int seg = 0;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+    while (i >= runs.start[seg + 1]) ++seg;
+    while (i < runs.start[seg]) --seg;
+    float4* v = reinterpret_cast<float4*>(static_cast<char*>(runs.ptr[seg]) + (i - runs.start[seg]) * (kHeadDim * 4));
+    for (int w = 0; w < words; ++w) {
+      float4 x = v[w];
+      const int p0 = 2 * w, p1 = 2 * w + 1;
+      const float a0 = x.x * tab.c[p0] - x.y * tab.s[p0], b0 = x.x * tab.s[p0] + x.y * tab.c[p0];
+      x.x = a0;
+      x.y = b0;
+      if (p1 < tab.pairs) {
+        const float a1 = x.z * tab.c[p1] - x.w * tab.s[p1], b1 = x.z * tab.s[p1] + x.w * tab.c[p1];
+        x.z = a1;
+        x.w = b1;
+      }
+      v[w] = x;
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_rope_shift_f32(const RowRuns& runs, const RopeTable& tab, cudaStream_t st) {
+  const long long total = runs.start[runs.n];
+  if (total <= 0 || tab.pairs <= 0) return cudaSuccess;
+  const long long want = (total + 255) / 256;
+  const int grid = static_cast<int>(want < 4096 ? want : 4096);
+  rope_shift_f32_kernel<<<grid, 256, 0, st>>>(runs, tab);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_rope_shift(const RowRuns& runs, const RopeTable& tab, cudaStream_t st) {
   const long long total = runs.start[runs.n];

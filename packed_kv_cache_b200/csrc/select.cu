@@ -6,7 +6,12 @@
 // archived (PackForcing (arXiv), "Compressed Mid Tokens").  Summed over a
 // block's keys and averaged over heads this is
 //   S[b, p] = sum_{j, h, d} qsum[b, h, d] * Kc[b, p, j, h, d] / (n n_c H sqrt(D)),
-// qsum = sum of the block's queries.  Two kernels, both HBM streams:
+// qsum = sum of the block's queries.  By linearity this is also
+//   S[b, p] = qsum[b] . kbar[b, p] / (n H sqrt(D)),  kbar = the block's mean key,
+// so when the cache keeps each compressed block's mean key (computed once,
+// when the block enters the pool) scoring reads 6 KB per block instead of its
+// n_c keys (score_mean_kernel).  Otherwise (the allocation-free entry point)
+// two HBM-streaming kernels:
 //   1. qpool: 32-row chunks of Q summed per column, added into qsum[b].
 //   2. score: one CTA per 32-row chunk of a pool block, a dot product with
 //      qsum[b]; the last CTA of batch item b (ticket counter) sums the
@@ -111,62 +116,13 @@ __device__ unsigned block_exclusive_scan(unsigned v, unsigned* total) {
   return before + x - v;
 }
 
-__global__ void __launch_bounds__(kThreads, 5) score_kernel(const SelectArgs a) {
-  extern __shared__ float smem[];
-  float* qs = smem;                                      // [HD]
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + a.HD);  // [count]
-  __shared__ float red[kThreads / 32];
-  __shared__ unsigned is_last;
+// The last CTA of batch item b: block scores from the partial sums, exact
+// radix selection of the n_top largest (ties to the older block), outputs in
+// ascending age, and the cleanup that leaves qsum[b] and ticket[b] zero.
+__device__ void select_tail(const SelectArgs& a, int b, uint32_t* keys) {
   __shared__ unsigned hist[256];
   __shared__ unsigned sh_prefix, sh_need;
-
-  const int b = blockIdx.y;
-  const int p = blockIdx.x / a.chunks_per_block;
-  const int c = blockIdx.x % a.chunks_per_block;
   const int t = threadIdx.x;
-  const int G = a.HD / 8;
-
-  for (int i = t; i < a.HD; i += kThreads) qs[i] = a.qsum[static_cast<long long>(b) * a.HD + i];
-  __syncthreads();
-
-  const int slot = (a.head + p) % a.slots;
-  const int row_lo = c * a.chunk_rows;
-  const int rows = min(a.n_c, row_lo + a.chunk_rows) - row_lo;
-  const uint4* K = static_cast<const uint4*>(a.pool_k) +
-                   ((static_cast<long long>(b) * a.slots + slot) * a.n_c + row_lo) * G;
-  const int nu = rows * G;
-  float acc = 0.f;
-  constexpr int U = 6;
-  for (int u0 = t; u0 < nu; u0 += kThreads * U) {
-    uint4 w[U];
-#pragma unroll
-    for (int k = 0; k < U; ++k) {
-      const int u = u0 + k * kThreads;
-      if (u < nu) w[k] = __ldg(K + u);
-    }
-#pragma unroll
-    for (int k = 0; k < U; ++k) {
-      const int u = u0 + k * kThreads;
-      if (u < nu) acc += dot_bf16x8(w[k], qs + (u % G) * 8);
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  if ((t & 31) == 0) red[t >> 5] = acc;
-  __syncthreads();
-  if (t == 0) {
-    float s = 0.f;
-    for (int k = 0; k < kThreads / 32; ++k) s += red[k];
-    a.partial[(static_cast<long long>(b) * a.slots + p) * a.chunks_per_block + c] = s;
-    __threadfence();
-    const unsigned total = static_cast<unsigned>(a.count * a.chunks_per_block);
-    is_last = (atomicAdd(&a.ticket[b], 1u) == total - 1u) ? 1u : 0u;
-  }
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-
-  // ---- last CTA of batch item b: block scores, top-k, cleanup
   const int count = a.count;
   for (int q = t; q < count; q += kThreads) {
     const float* pp = a.partial + (static_cast<long long>(b) * a.slots + q) * a.chunks_per_block;
@@ -239,6 +195,113 @@ __global__ void __launch_bounds__(kThreads, 5) score_kernel(const SelectArgs a) 
   if (t == 0) a.ticket[b] = 0u;
 }
 
+__global__ void __launch_bounds__(kThreads, 5) score_kernel(const SelectArgs a) {
+  extern __shared__ float smem[];
+  float* qs = smem;                                      // [HD]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + a.HD);  // [count]
+  __shared__ float red[kThreads / 32];
+  __shared__ unsigned is_last;
+
+  const int b = blockIdx.y;
+  const int p = blockIdx.x / a.chunks_per_block;
+  const int c = blockIdx.x % a.chunks_per_block;
+  const int t = threadIdx.x;
+  const int G = a.HD / 8;
+
+  for (int i = t; i < a.HD; i += kThreads) qs[i] = a.qsum[static_cast<long long>(b) * a.HD + i];
+  __syncthreads();
+
+  const int slot = (a.head + p) % a.slots;
+  const int row_lo = c * a.chunk_rows;
+  const int rows = min(a.n_c, row_lo + a.chunk_rows) - row_lo;
+  const uint4* K = static_cast<const uint4*>(a.pool_k) +
+                   ((static_cast<long long>(b) * a.slots + slot) * a.n_c + row_lo) * G;
+  const int nu = rows * G;
+  float acc = 0.f;
+  constexpr int U = 6;
+  for (int u0 = t; u0 < nu; u0 += kThreads * U) {
+    uint4 w[U];
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      const int u = u0 + k * kThreads;
+      if (u < nu) w[k] = __ldg(K + u);
+    }
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      const int u = u0 + k * kThreads;
+      if (u < nu) acc += dot_bf16x8(w[k], qs + (u % G) * 8);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((t & 31) == 0) red[t >> 5] = acc;
+  __syncthreads();
+  if (t == 0) {
+    float s = 0.f;
+    for (int k = 0; k < kThreads / 32; ++k) s += red[k];
+    a.partial[(static_cast<long long>(b) * a.slots + p) * a.chunks_per_block + c] = s;
+    __threadfence();
+    const unsigned total = static_cast<unsigned>(a.count * a.chunks_per_block);
+    is_last = (atomicAdd(&a.ticket[b], 1u) == total - 1u) ? 1u : 0u;
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+
+  select_tail(a, b, keys);
+}
+
+// Factored scoring: S[b, p] = qsum[b] . kbar[b, slot(p)] * scale, one warp per
+// block, kbar the block's mean key (float32, kept with the pool).
+__global__ void __launch_bounds__(kThreads) score_mean_kernel(const SelectArgs a) {
+  extern __shared__ float smem[];
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem);  // [count], used by the last CTA
+  __shared__ unsigned is_last;
+  const int b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int p = blockIdx.x * (kThreads / 32) + warp;
+  if (p < a.count) {
+    const int slot = (a.head + p) % a.slots;
+    const float4* q = reinterpret_cast<const float4*>(a.qsum + static_cast<long long>(b) * a.HD);
+    const float4* k = reinterpret_cast<const float4*>(a.kbar + (static_cast<long long>(b) * a.slots + slot) * a.HD);
+    float acc = 0.f;
+    for (int i = lane; i < a.HD / 4; i += 32) {
+      const float4 x = q[i], y = __ldg(k + i);
+      acc = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, acc))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) a.partial[static_cast<long long>(b) * a.slots + p] = acc;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    is_last = (atomicAdd(&a.ticket[b], 1u) == gridDim.x - 1u) ? 1u : 0u;
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  select_tail(a, b, keys);
+}
+
+// kbar[b, slot] = mean over the block's n_c keys, for slots [slot0, slot0 + gridDim.x).
+__global__ void __launch_bounds__(kThreads) kmean_kernel(const void* pool_k, float* kbar, int slots, int n_c,
+                                                         int HD, int slot0) {
+  const int b = blockIdx.y;
+  const int slot = slot0 + blockIdx.x;
+  const int G = HD / 8;
+  const uint4* K = static_cast<const uint4*>(pool_k) + (static_cast<long long>(b) * slots + slot) * n_c * G;
+  float4* out = reinterpret_cast<float4*>(kbar + (static_cast<long long>(b) * slots + slot) * HD);
+  const float inv = 1.f / static_cast<float>(n_c);
+  for (int g = threadIdx.x; g < G; g += kThreads) {
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll 4
+    for (int r = 0; r < n_c; ++r) acc_bf16x8(acc, __ldg(K + static_cast<long long>(r) * G + g));
+    out[2 * g] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    out[2 * g + 1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
@@ -247,6 +310,17 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
   qpool_kernel<<<g1, kThreads, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (a.kbar != nullptr) {
+    // factored: one warp per block against its cached mean key
+    const size_t smem = static_cast<size_t>(a.count) * 4;
+    if (smem > 48 * 1024) {
+      e = cudaFuncSetAttribute(score_mean_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+    }
+    dim3 g2((a.count + kThreads / 32 - 1) / (kThreads / 32), a.B);
+    score_mean_kernel<<<g2, kThreads, smem, st>>>(a);
+    return cudaGetLastError();
+  }
   const size_t smem = static_cast<size_t>(a.HD) * 4 + static_cast<size_t>(a.count) * 4;
   if (smem > 48 * 1024) {
     e = cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -254,6 +328,13 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
   }
   dim3 g2(a.count * a.chunks_per_block, a.B);
   score_kernel<<<g2, kThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kmean(const void* pool_k, float* kbar, int B, int slots, int n_c, int HD, int slot0, int nslots,
+                         cudaStream_t st) {
+  if (nslots <= 0) return cudaSuccess;
+  kmean_kernel<<<dim3(nslots, B), kThreads, 0, st>>>(pool_k, kbar, slots, n_c, HD, slot0);
   return cudaGetLastError();
 }
 
@@ -354,6 +435,7 @@ extern "C" pf_status pf_select_mid_static(const void* Q, int batch, int n, int h
   a.HD = HD;
   a.qsum = sc->qsum;
   a.pool_k = pool_k;
+  a.kbar = nullptr;   // no cached mean keys: stream the pool
   a.slots = pool_slots;
   a.n_c = n_c;
   a.head = head;

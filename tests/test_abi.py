@@ -61,7 +61,8 @@ def test_cache_bytes_layout(pf):
     slots = wl.mid_capacity + wl.recent_blocks
     cpb = (182 + 31) // 32
     per_layer = (2 * (al(2 * 6240 * row) + al(slots * 182 * row) + al(6240 * row))
-                 + al(16 * 4) + al(slots * 4) + al(slots * cpb * 4) + al(12 * 128 * 4) + al(4))
+                 + al(16 * 4) + al(slots * 4) + al(slots * cpb * 4) + al(12 * 128 * 4) + al(4)
+                 + al(slots * 1536 * 4))   # mean key of every pool slot
     # shared attention scratch: 256 split-tail slots of 128x128 fp32 partial
     # outputs, their row max / row sum, and 256 tickets
     scratch = 256 * 128 * 128 * 4 + 256 * 2 * 128 * 4 + 256 * 4

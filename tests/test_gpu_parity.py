@@ -146,6 +146,32 @@ def test_selection_bit_exact(pf, name):
     assert torch.equal(sel, sel2)
 
 
+@pytest.mark.parametrize("name", ["ragged_b", "layer"])
+def test_selection_after_rotating_the_pool(pf, name):
+    # selection scores the blocks' cached mean keys; a RoPE shift of the mid
+    # pool must rotate them with the keys
+    wl = _wl(name)
+    d = synth.make_layer(wl, seed_for(name))
+    cache = build_cache(pf, wl, d)
+    delta = 3 * d["delta"] + 1
+    cache.rope_shift(0, pf.PART_MID | pf.PART_RECENT, delta)
+    B, P = wl.batch, wl.pool_blocks
+    k = min(wl.n_top, P)
+    sel = torch.full((B, k), -1, dtype=torch.int32, device="cuda")
+    sc = torch.zeros((B, P), dtype=torch.float32, device="cuda")
+    cache.select_mid(0, d["Q"].cuda(), sel, sc)
+    torch.cuda.synchronize()
+    midK = oracle.round_bf16(oracle.rope_shift(d["mid_K"], delta))
+    S_ref = oracle.select_scores(d["Q"], midK)
+    scale = np.abs(S_ref).max(axis=1, keepdims=True)
+    assert np.max(np.abs(sc.cpu().numpy() - S_ref) / scale) < 1e-3
+    margin = oracle.selection_margin(S_ref, wl.n_top)
+    sel_ref = oracle.select_topk(S_ref, wl.n_top)
+    for b in range(B):
+        if margin[b] >= 1e-3:
+            assert np.array_equal(sel.cpu().numpy()[b], sel_ref[b])
+
+
 def test_selection_ties_go_to_older_blocks(pf):
     wl = _wl("ragged_a").replace(pool_blocks=9, planted=0, mid_capacity=9, n_top=4)
     d = synth.make_layer(wl, 5)
