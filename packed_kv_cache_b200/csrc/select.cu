@@ -71,8 +71,17 @@ __global__ void __launch_bounds__(kThreads) qpool_kernel(const SelectArgs a) {
     const int g = g0 + gl;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (r0 < rstep && g < G) {
-#pragma unroll 4
-      for (int r = row_lo + r0; r < row_hi; r += rstep) acc_bf16x8(acc, Q[static_cast<long long>(r) * G + g]);
+      // eight rows in flight per step
+      for (int r = row_lo + r0; r < row_hi; r += 8 * rstep) {
+        uint4 w[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int rr = r + k * rstep;
+          w[k] = rr < row_hi ? __ldg(Q + static_cast<long long>(rr) * G + g) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc_bf16x8(acc, w[k]);
+      }
     }
 #pragma unroll
     for (int e = 0; e < 8; ++e) red[t * 8 + e] = acc[e];
@@ -284,21 +293,37 @@ __global__ void __launch_bounds__(kThreads) score_mean_kernel(const SelectArgs a
   select_tail(a, b, keys);
 }
 
-// kbar[b, slot] = mean over the block's n_c keys, for slots [slot0, slot0 + gridDim.x).
+// kbar[b, slot] = mean over the block's n_c keys.  CTA (slot, b, z): 32
+// column groups (16 bytes each) starting at group 32 z, rows split over the 8
+// warps; grid.x covers slots [slot0, slot0 + gridDim.x).
 __global__ void __launch_bounds__(kThreads) kmean_kernel(const void* pool_k, float* kbar, int slots, int n_c,
                                                          int HD, int slot0) {
+  __shared__ float red[kThreads / 32][32][9];
   const int b = blockIdx.y;
   const int slot = slot0 + blockIdx.x;
   const int G = HD / 8;
+  const int lane = threadIdx.x & 31, phase = threadIdx.x >> 5;
+  const int g = blockIdx.z * 32 + lane;
   const uint4* K = static_cast<const uint4*>(pool_k) + (static_cast<long long>(b) * slots + slot) * n_c * G;
-  float4* out = reinterpret_cast<float4*>(kbar + (static_cast<long long>(b) * slots + slot) * HD);
-  const float inv = 1.f / static_cast<float>(n_c);
-  for (int g = threadIdx.x; g < G; g += kThreads) {
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if (g < G) {
 #pragma unroll 4
-    for (int r = 0; r < n_c; ++r) acc_bf16x8(acc, __ldg(K + static_cast<long long>(r) * G + g));
-    out[2 * g] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-    out[2 * g + 1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+    for (int r = phase; r < n_c; r += kThreads / 32) acc_bf16x8(acc, __ldg(K + static_cast<long long>(r) * G + g));
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) red[phase][lane][e] = acc[e];
+  __syncthreads();
+  if (phase == 0 && g < G) {
+    const float inv = 1.f / static_cast<float>(n_c);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float s = 0.f;
+      for (int k = 0; k < kThreads / 32; ++k) s += red[k][lane][e];
+      acc[e] = s * inv;
+    }
+    float4* out = reinterpret_cast<float4*>(kbar + (static_cast<long long>(b) * slots + slot) * HD) + 2 * g;
+    out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
 }
 
@@ -334,7 +359,7 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
 cudaError_t launch_kmean(const void* pool_k, float* kbar, int B, int slots, int n_c, int HD, int slot0, int nslots,
                          cudaStream_t st) {
   if (nslots <= 0) return cudaSuccess;
-  kmean_kernel<<<dim3(nslots, B), kThreads, 0, st>>>(pool_k, kbar, slots, n_c, HD, slot0);
+  kmean_kernel<<<dim3(nslots, B, (HD / 8 + 31) / 32), kThreads, 0, st>>>(pool_k, kbar, slots, n_c, HD, slot0);
   return cudaGetLastError();
 }
 
