@@ -12,12 +12,13 @@
 // when the block enters the pool) scoring reads 6 KB per block instead of its
 // n_c keys (score_mean_kernel).  Otherwise (the allocation-free entry point)
 // two HBM-streaming kernels:
-//   1. qpool: 32-row chunks of Q summed per column, added into qsum[b].
+//   1. qpool: the columns of Q[b] summed over the block's rows into qsum[b]
+//      (shared by both paths).
 //   2. score: one CTA per 32-row chunk of a pool block, a dot product with
 //      qsum[b]; the last CTA of batch item b (ticket counter) sums the
 //      chunks of each block in a fixed order, runs an exact radix select of
 //      the n_top largest scores (ties to the older block), writes the
-//      selection in ascending age, and clears qsum[b] and its ticket.
+//      selection in ascending age, and clears its ticket.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -55,46 +56,55 @@ __device__ __forceinline__ float dot_bf16x8(const uint4& w, const float* q) {
   return s;
 }
 
-// qsum[b, :] += column sums of Q rows [32 c, 32 c + 32) of batch item b.
-__global__ void __launch_bounds__(kThreads) qpool_kernel(const SelectArgs a) {
+// qsum[b] = column sums of Q[b] (the block's n queries).  CTA (x, b) owns
+// the 16-byte column groups [2x, 2x + 2) (one 32-byte sector of every row)
+// and sums them over all n rows of batch item b: no atomics, qsum[b] is
+// written, not accumulated.
+// kQcPhases row phases, each thread keeps kQcLoads row loads in flight; two
+// CTAs per SM.
+constexpr int kQcThreads = 512;
+constexpr int kQcPhases = kQcThreads / 2;
+constexpr int kQcLoads = 6;   // row loads in flight per thread
+__global__ void __launch_bounds__(kQcThreads, 2) qpool_kernel(const SelectArgs a) {
   const int b = blockIdx.y;
-  const int G = a.HD / 8;                        // 16-byte groups per row
-  const int Gp = G < kThreads ? G : kThreads;    // groups handled per pass
-  const int rstep = kThreads / Gp;               // row phases per pass
+  const int G = a.HD / 8;
   const int t = threadIdx.x;
-  const int r0 = t / Gp, gl = t % Gp;
-  const int row_lo = blockIdx.x * 32;
-  const int row_hi = min(a.n, row_lo + 32);
-  __shared__ float red[kThreads * 8];
-  const uint4* Q = static_cast<const uint4*>(a.Q) + static_cast<long long>(b) * a.n * G;
-  for (int g0 = 0; g0 < G; g0 += Gp) {
-    const int g = g0 + gl;
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    if (r0 < rstep && g < G) {
-      // eight rows in flight per step
-      for (int r = row_lo + r0; r < row_hi; r += 8 * rstep) {
-        uint4 w[8];
+  const int g = blockIdx.x * 2 + (t & 1);
+  const int phase = t >> 1;
+  const uint4* Q = static_cast<const uint4*>(a.Q) + static_cast<long long>(b) * a.n * G + g;
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if (g < G) {
+    const long long stride = static_cast<long long>(kQcPhases) * G;
+    const uint4* q = Q + static_cast<long long>(phase) * G;
+    for (int r = phase; r < a.n; r += kQcLoads * kQcPhases, q += kQcLoads * stride) {
+      uint4 w[kQcLoads];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int rr = r + k * rstep;
-          w[k] = rr < row_hi ? __ldg(Q + static_cast<long long>(rr) * G + g) : make_uint4(0u, 0u, 0u, 0u);
-        }
+      for (int k = 0; k < kQcLoads; ++k)
+        w[k] = r + k * kQcPhases < a.n ? __ldg(q + k * stride) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) acc_bf16x8(acc, w[k]);
-      }
+      for (int k = 0; k < kQcLoads; ++k) acc_bf16x8(acc, w[k]);
     }
+  }
+  // reduce the row phases: warp shuffles over the 16 phases of a warp, then
+  // the 16 warps' partials through shared memory
 #pragma unroll
-    for (int e = 0; e < 8; ++e) red[t * 8 + e] = acc[e];
-    __syncthreads();
-    if (r0 == 0 && g < G) {
+  for (int e = 0; e < 8; ++e) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        float s = red[t * 8 + e];
-        for (int k = 1; k < rstep; ++k) s += red[(k * Gp + gl) * 8 + e];
-        atomicAdd(&a.qsum[static_cast<long long>(b) * a.HD + g * 8 + e], s);
-      }
-    }
-    __syncthreads();
+    for (int off = 2; off < 32; off <<= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+  }
+  __shared__ float red[kQcThreads / 32][2][8];
+  const int lane = t & 31, warp = t >> 5;
+  if (lane < 2) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[warp][lane][e] = acc[e];
+  }
+  __syncthreads();
+  if (t < 16) {
+    const int col = t >> 3, e = t & 7;
+    float s = 0.f;
+    for (int w = 0; w < kQcThreads / 32; ++w) s += red[w][col][e];
+    const int gg = blockIdx.x * 2 + col;
+    if (gg < G) a.qsum[static_cast<long long>(b) * a.HD + gg * 8 + e] = s;
   }
 }
 
@@ -127,7 +137,7 @@ __device__ unsigned block_exclusive_scan(unsigned v, unsigned* total) {
 
 // The last CTA of batch item b: block scores from the partial sums, exact
 // radix selection of the n_top largest (ties to the older block), outputs in
-// ascending age, and the cleanup that leaves qsum[b] and ticket[b] zero.
+// ascending age, and the cleanup that leaves ticket[b] zero.
 __device__ void select_tail(const SelectArgs& a, int b, uint32_t* keys) {
   __shared__ unsigned hist[256];
   __shared__ unsigned sh_prefix, sh_need;
@@ -154,9 +164,18 @@ __device__ void select_tail(const SelectArgs& a, int b, uint32_t* keys) {
       hist[t] = 0u;
       __syncthreads();
       const unsigned pre = sh_prefix;
-      for (int q = t; q < count; q += kThreads) {
-        const uint32_t key = keys[q];
-        if (shift == 24 || (key >> (shift + 8)) == (pre >> (shift + 8))) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      // warp-aggregated: one shared-memory atomic per distinct digit per warp
+      // (the keys' leading digits are mostly equal)
+      for (int q0 = 0; q0 < count; q0 += kThreads) {
+        const int q = q0 + t;
+        const uint32_t key = q < count ? keys[q] : 0u;
+        const bool take = q < count && (shift == 24 || (key >> (shift + 8)) == (pre >> (shift + 8)));
+        const unsigned digit = (key >> shift) & 255u;
+        const unsigned m = __ballot_sync(0xffffffffu, take);
+        if (take) {
+          const unsigned grp = __match_any_sync(m, digit);
+          if ((t & 31) == __ffs(grp) - 1) atomicAdd(&hist[digit], static_cast<unsigned>(__popc(grp)));
+        }
       }
       __syncthreads();
       {
@@ -200,7 +219,6 @@ __device__ void select_tail(const SelectArgs& a, int b, uint32_t* keys) {
       ++pos;
     }
   }
-  for (int i = t; i < a.HD; i += kThreads) a.qsum[static_cast<long long>(b) * a.HD + i] = 0.f;
   if (t == 0) a.ticket[b] = 0u;
 }
 
@@ -264,19 +282,36 @@ __global__ void __launch_bounds__(kThreads, 5) score_kernel(const SelectArgs a) 
 // block, kbar the block's mean key (float32, kept with the pool).
 __global__ void __launch_bounds__(kThreads) score_mean_kernel(const SelectArgs a) {
   extern __shared__ float smem[];
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem);  // [count], used by the last CTA
+  float* qs = smem;                                           // [HD] qsum[b]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + a.HD);  // [count], used by the last CTA
   __shared__ unsigned is_last;
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int p = blockIdx.x * (kThreads / 32) + warp;
+  for (int i = threadIdx.x; i < a.HD; i += kThreads) qs[i] = a.qsum[static_cast<long long>(b) * a.HD + i];
+  __syncthreads();
   if (p < a.count) {
     const int slot = (a.head + p) % a.slots;
-    const float4* q = reinterpret_cast<const float4*>(a.qsum + static_cast<long long>(b) * a.HD);
+    const float4* q = reinterpret_cast<const float4*>(qs);
     const float4* k = reinterpret_cast<const float4*>(a.kbar + (static_cast<long long>(b) * a.slots + slot) * a.HD);
+    const int nv = a.HD / 4;
     float acc = 0.f;
-    for (int i = lane; i < a.HD / 4; i += 32) {
-      const float4 x = q[i], y = __ldg(k + i);
-      acc = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, acc))));
+    // eight 16-byte loads of the mean key in flight per lane
+    for (int i0 = lane; i0 < nv; i0 += 32 * 8) {
+      float4 y[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + 32 * u;
+        y[u] = i < nv ? __ldg(k + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + 32 * u;
+        if (i < nv) {
+          const float4 x = q[i];
+          acc = fmaf(x.x, y[u].x, fmaf(x.y, y[u].y, fmaf(x.z, y[u].z, fmaf(x.w, y[u].w, acc))));
+        }
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -331,13 +366,13 @@ __global__ void __launch_bounds__(kThreads) kmean_kernel(const void* pool_k, flo
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
   if (a.count <= 0) return cudaSuccess;
-  dim3 g1((a.n + 31) / 32, a.B);
-  qpool_kernel<<<g1, kThreads, 0, st>>>(a);
+  dim3 g1((a.HD / 8 + 1) / 2, a.B);
+  qpool_kernel<<<g1, kQcThreads, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (a.kbar != nullptr) {
     // factored: one warp per block against its cached mean key
-    const size_t smem = static_cast<size_t>(a.count) * 4;
+    const size_t smem = static_cast<size_t>(a.HD) * 4 + static_cast<size_t>(a.count) * 4;
     if (smem > 48 * 1024) {
       e = cudaFuncSetAttribute(score_mean_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
       if (e != cudaSuccess) return e;
