@@ -37,7 +37,9 @@ sys.path.insert(0, ROOT)
 
 WORKLOAD = "layer"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-LAUNCHES_PER_STEP = 5          # qpool, score+top-k, attend, append copy, rope shift
+# library kernels per step: qpool + score_mean (select), attend, copy_runs +
+# kmean (append with a compressed copy), and rope_shift when a block was evicted
+LAUNCHES_PER_STEP_BASE = 5
 
 
 # ---------------------------------------------------------------- distributed plumbing
@@ -235,6 +237,7 @@ def run_gpu(args):
         ev = cache.append_block(0, k, v, kc, vc)
         if ev:
             cache.rope_shift(0, pf.PART_SINK, ev * wl.block_frames)
+        return LAUNCHES_PER_STEP_BASE + (1 if ev else 0)
 
     clocks = ClockSampler(local)
     clocks.start()
@@ -253,10 +256,11 @@ def run_gpu(args):
     torch.cuda.synchronize(dev)
     barrier()
     t_start = time.time()
+    launches = 0
     for i in range(args.steps):
         flush(i + 7)
         ev_step[i][0].record(stream)
-        step(Q, Kn, Vn, Kcn, Vcn, O, ev_att[i])
+        launches += step(Q, Kn, Vn, Kcn, Vcn, O, ev_att[i])
         ev_step[i][1].record(stream)
     torch.cuda.synchronize(dev)
     t_end = time.time()
@@ -337,7 +341,7 @@ def run_gpu(args):
         },
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / args.steps, 4)},
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": launches,
         "clocks": clk,
     }
     if rank == 0 and not args.no_cpu_baseline:
@@ -375,12 +379,17 @@ def oracle_step(d, wl, rows):
 def cpu_baseline(d, wl, budget_s=15.0):
     import numpy as np
     dc = {k: (v.cpu() if hasattr(v, "cpu") else v) for k, v in d.items()}
-    rows = np.arange(16)
-    t0 = time.perf_counter()
-    fl = oracle_step(dc, wl, rows)
-    dt = time.perf_counter() - t0
-    # grow the sample toward the budget
-    nrows = int(min(wl.n, max(16, 16 * budget_s / max(dt, 1e-3) * 0.8)))
+    # two short calibrations separate the fixed cost (selection over the
+    # pool, sink shift) from the per-query-row cost of the attention sample
+    times = []
+    for nr in (16, 64):
+        rows = np.linspace(0, wl.n - 1, nr).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle_step(dc, wl, rows)
+        times.append(time.perf_counter() - t0)
+    per_row = max((times[1] - times[0]) / 48, 1e-6)
+    fixed = max(times[0] - 16 * per_row, 0.0)
+    nrows = int(min(wl.n, max(16, (0.9 * budget_s - fixed) / per_row)))
     rows = np.linspace(0, wl.n - 1, nrows).astype(np.int64)
     t0 = time.perf_counter()
     fl = oracle_step(dc, wl, rows)
@@ -591,7 +600,7 @@ def run_suite(args):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--ref-rows", type=int, default=24)
