@@ -178,6 +178,53 @@ pf_status pf_select_mid(pf_cache* cache, int layer, const void* Q, int32_t* sel_
                         float* scores_out, void* stream);
 
 /*
+ * Routing policies and options of pf_select_mid_ex.
+ *
+ * PF_ROUTE_SCORE (the method): the scores above, optionally over a subset of
+ *   the queries and heads.  The digest's limitations paragraph says the
+ *   selection subsamples the query tokens and uses half of the attention
+ *   heads to stay cheap; the pages give neither the sampling rule nor which
+ *   half, so both are options: query rows 0, q_stride, 2 q_stride, ... and
+ *   heads [head_lo, head_hi).  With heads_total > 0 the score is divided by
+ *   heads_total instead of the number of heads used, so scores computed on
+ *   disjoint head ranges (for example by GPUs that each hold some of the
+ *   heads) add up to the all-head score.
+ * PF_ROUTE_SCORES_ONLY: the same scores into scores_out (required), no
+ *   top-k and no stored selection (the partial scores of a head shard).
+ * PF_ROUTE_GIVEN: top-k of caller-provided scores (scores_in, device,
+ *   [B, mid_count] float by age): random routing (random scores; PackForcing
+ *   (arXiv), "FIFO vs. Dynamic Context Selection", the random baseline), or
+ *   the sum of head shards' partial scores.  Same ranking rule and outputs as
+ *   PF_ROUTE_SCORE.
+ * PF_ROUTE_FIFO: the n_top most recent live blocks (the FIFO baseline of the
+ *   same table: chronological retention, no scoring).  Reads no scores.
+ */
+#define PF_ROUTE_SCORE 0
+#define PF_ROUTE_SCORES_ONLY 1
+#define PF_ROUTE_GIVEN 2
+#define PF_ROUTE_FIFO 3
+
+typedef struct pf_select_opts {
+  int policy;             /* PF_ROUTE_* */
+  int q_stride;           /* >= 1; 1 = every query row */
+  int head_lo, head_hi;   /* heads used by the score; head_hi = 0 means all */
+  int heads_total;        /* score divisor in heads; 0 = the heads used */
+  const float* scores_in; /* PF_ROUTE_GIVEN only */
+} pf_select_opts;
+
+/*
+ * pf_select_mid with a routing policy (see above).  opts NULL = the method's
+ * defaults (PF_ROUTE_SCORE, every query row, every head) = pf_select_mid.
+ * sel_out / scores_out as for pf_select_mid (scores_out is required for
+ * PF_ROUTE_SCORES_ONLY and ignored by PF_ROUTE_FIFO).  PF_ROUTE_SCORE and
+ * PF_ROUTE_SCORES_ONLY launch two kernels, PF_ROUTE_GIVEN and PF_ROUTE_FIFO
+ * one.  Errors: PF_ERR_ARG for a bad policy, stride, head range, or a
+ * missing scores_in / scores_out.
+ */
+pf_status pf_select_mid_ex(pf_cache* cache, int layer, const void* Q, const pf_select_opts* opts,
+                           int32_t* sel_out, float* scores_out, void* stream);
+
+/*
  * Incremental temporal RoPE adjustment (PackForcing (arXiv), "Incremental
  * RoPE adjustment"; digest, method step (4)): multiply the stored keys'
  * temporal rotary pairs by e^{i theta_t,k delta},

@@ -41,7 +41,7 @@ import numpy as np
 __all__ = [
     "token_counts", "dense_context_tokens", "kv_bytes",
     "rope_thetas", "rope_encode", "rope_shift",
-    "select_scores", "select_scores_bruteforce", "select_topk", "selection_margin",
+    "select_scores", "select_scores_bruteforce", "select_topk", "selection_margin", "select_fifo",
     "attend", "attend_loops", "merge_partials", "cache_partitions",
     "to_f64", "round_bf16",
 ]
@@ -192,7 +192,7 @@ def rope_shift(keys, delta, split=(44, 42, 42), base: float = 10000.0) -> np.nda
 # dynamic top-k context selection
 # --------------------------------------------------------------------------
 
-def select_scores(Q, pool_K) -> np.ndarray:
+def select_scores(Q, pool_K, q_stride: int = 1, heads=None, heads_norm=None) -> np.ndarray:
     """Block scores S[b, p] = (1/H) sum_h qbar_{b,h} . kbar_{b,p,h} / sqrt(d_h).
 
     Q: [B, n, H, D] current-block queries.  pool_K: [B, P, n_c, H, D], the
@@ -200,13 +200,33 @@ def select_scores(Q, pool_K) -> np.ndarray:
     digest's phi_j = sum_i q_i^T k_j / sqrt(d) (step (3)) summed over the
     block's keys and averaged over heads, divided by n * n_c (the ranking is
     unchanged).
+
+    The digest's limitations paragraph says the selection subsamples the
+    query tokens and uses half of the heads to stay cheap, without saying
+    how; the options read that as: queries 0, q_stride, 2 q_stride, ... only;
+    heads [lo, hi) only (heads = (lo, hi)); and the head sum divided by
+    heads_norm (default: the number of heads used), so that scores of
+    disjoint head ranges divided by the total head count add up to the
+    all-head score.
     """
-    q = to_f64(Q)
+    q = to_f64(Q)[:, ::q_stride]
     k = to_f64(pool_K)
-    H, D = q.shape[2], q.shape[3]
-    qbar = q.mean(axis=1)                         # [B, H, D]
-    kbar = k.mean(axis=2)                         # [B, P, H, D]
-    return np.einsum("bhd,bphd->bp", qbar, kbar) / (H * math.sqrt(D))
+    lo, hi = heads if heads is not None else (0, q.shape[2])
+    q = q[:, :, lo:hi]
+    k = k[:, :, :, lo:hi]
+    D = q.shape[3]
+    Hn = heads_norm if heads_norm else hi - lo
+    qbar = q.mean(axis=1)                         # [B, H', D]
+    kbar = k.mean(axis=2)                         # [B, P, H', D]
+    return np.einsum("bhd,bphd->bp", qbar, kbar) / (Hn * math.sqrt(D))
+
+
+def select_fifo(count: int, n_top: int) -> np.ndarray:
+    """FIFO routing: the min(n_top, count) most recent of `count` live blocks,
+    ascending age (PackForcing (arXiv), "FIFO vs. Dynamic Context Selection":
+    chronological retention, the baseline of dynamic selection)."""
+    k = min(n_top, count)
+    return np.arange(count - k, count, dtype=np.int64)
 
 
 def select_scores_bruteforce(Q, pool_K) -> np.ndarray:

@@ -21,7 +21,8 @@ __all__ = [
     "lib", "library_path", "pf_version", "pf_cache_bytes", "pf_cache_create", "pf_cache_destroy",
     "pf_cache_layer_info", "pf_cache_append_block", "pf_cache_load_mid", "pf_select_mid",
     "pf_rope_shift", "pf_attend", "pf_poll_device_error", "pf_selftest_wait_timeout",
-    "pf_select_mid_static",
+    "pf_select_mid_static", "pf_select_mid_ex", "SelectOpts",
+    "ROUTE_SCORE", "ROUTE_SCORES_ONLY", "ROUTE_GIVEN", "ROUTE_FIFO",
     "PackedKVCache", "config_for",
 ]
 
@@ -29,6 +30,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libpf.so")
 
 PART_SINK, PART_MID, PART_RECENT = 1, 2, 4
+ROUTE_SCORE, ROUTE_SCORES_ONLY, ROUTE_GIVEN, ROUTE_FIFO = 0, 1, 2, 3
 STATUS = {0: "PF_OK", 1: "PF_ERR_ARG", 2: "PF_ERR_ARENA", 3: "PF_ERR_STATE", 4: "PF_ERR_CAPACITY",
           5: "PF_ERR_CUDA", 6: "PF_ERR_TIMEOUT", 7: "PF_ERR_UNSUPPORTED"}
 
@@ -46,6 +48,11 @@ class Config(ctypes.Structure):
                 ("w", ctypes.c_int), ("sink_blocks", ctypes.c_int), ("recent_blocks", ctypes.c_int),
                 ("mid_capacity", ctypes.c_int), ("n_top", ctypes.c_int),
                 ("rope_split", ctypes.c_int * 3), ("rope_base", ctypes.c_float)]
+
+
+class SelectOpts(ctypes.Structure):
+    _fields_ = [("policy", ctypes.c_int), ("q_stride", ctypes.c_int), ("head_lo", ctypes.c_int),
+                ("head_hi", ctypes.c_int), ("heads_total", ctypes.c_int), ("scores_in", ctypes.c_void_p)]
 
 
 class LayerInfo(ctypes.Structure):
@@ -80,6 +87,7 @@ def _load():
         "pf_cache_append_block": ([vp, i32, vp, vp, vp, vp, ctypes.POINTER(i32), vp], i32),
         "pf_cache_load_mid": ([vp, i32, vp, vp, i32, ctypes.POINTER(i32), vp], i32),
         "pf_select_mid": ([vp, i32, vp, vp, vp, vp], i32),
+        "pf_select_mid_ex": ([vp, i32, vp, ctypes.POINTER(SelectOpts), vp, vp, vp], i32),
         "pf_rope_shift": ([vp, i32, u32, i32, vp], i32),
         "pf_attend": ([vp, i32, vp, vp, vp, vp, vp, vp], i32),
         "pf_poll_device_error": ([vp, vp, ctypes.POINTER(u32)], i32),
@@ -186,6 +194,19 @@ def pf_select_mid(handle, layer, Q, sel_out=None, scores_out=None, stream=None) 
                                               _dev(scores_out, "scores_out"), _stream(stream)))
 
 
+def pf_select_mid_ex(handle, layer, Q, policy=ROUTE_SCORE, q_stride=1, heads=None, heads_total=0,
+                     scores_in=None, sel_out=None, scores_out=None, stream=None) -> None:
+    """Selection with a routing policy: ROUTE_SCORE (the method, optionally on
+    every q_stride-th query row and the head range `heads` = (lo, hi)),
+    ROUTE_SCORES_ONLY (scores into scores_out, nothing stored), ROUTE_GIVEN
+    (top-k of scores_in), ROUTE_FIFO (the newest n_top blocks)."""
+    lo, hi = heads if heads is not None else (0, 0)
+    o = SelectOpts(policy, q_stride, lo, hi, heads_total, _dev(scores_in, "scores_in"))
+    _check("pf_select_mid_ex", lib.pf_select_mid_ex(handle, layer, _dev(Q, "Q"), ctypes.byref(o),
+                                                    _dev(sel_out, "sel_out"), _dev(scores_out, "scores_out"),
+                                                    _stream(stream)))
+
+
 def pf_rope_shift(handle, layer: int, parts: int, delta: int, stream=None) -> None:
     _check("pf_rope_shift", lib.pf_rope_shift(handle, layer, parts, delta, _stream(stream)))
 
@@ -247,6 +268,11 @@ class PackedKVCache:
 
     def select_mid(self, layer, Q, sel_out=None, scores_out=None, stream=None) -> None:
         pf_select_mid(self.handle, layer, Q, sel_out, scores_out, stream)
+
+    def select_mid_ex(self, layer, Q=None, policy=ROUTE_SCORE, q_stride=1, heads=None, heads_total=0,
+                      scores_in=None, sel_out=None, scores_out=None, stream=None) -> None:
+        pf_select_mid_ex(self.handle, layer, Q, policy, q_stride, heads, heads_total, scores_in, sel_out,
+                         scores_out, stream)
 
     def rope_shift(self, layer, parts, delta, stream=None) -> None:
         pf_rope_shift(self.handle, layer, parts, delta, stream)

@@ -496,16 +496,41 @@ pf_status pf_cache_load_mid(pf_cache* c, int layer, const void* Kc, const void* 
   return PF_OK;
 }
 
-pf_status pf_select_mid(pf_cache* c, int layer, const void* Q, int32_t* sel_out, float* scores_out, void* stream) {
+pf_status pf_select_mid_ex(pf_cache* c, int layer, const void* Q, const pf_select_opts* opts, int32_t* sel_out,
+                           float* scores_out, void* stream) {
   pf_status s = check_layer(c, layer);
   if (s != PF_OK) return s;
-  if ((s = check_ptr(Q, "Q")) != PF_OK) return s;
-  Layer& Ly = c->L[layer];
   const pf_config& cf = c->cfg;
   const Geometry& g = c->g;
-  if (Ly.mid_count == 0 || cf.n_top == 0) {
-    Ly.sel_valid = true;
-    Ly.n_sel = 0;
+  pf_select_opts o;
+  o.policy = PF_ROUTE_SCORE;
+  o.q_stride = 1;
+  o.head_lo = 0;
+  o.head_hi = 0;
+  o.heads_total = 0;
+  o.scores_in = nullptr;
+  if (opts != nullptr) o = *opts;
+  if (o.head_lo == 0 && o.head_hi == 0) o.head_hi = cf.heads;
+  if (o.policy < PF_ROUTE_SCORE || o.policy > PF_ROUTE_FIFO) return fail(PF_ERR_ARG, "unknown routing policy %d", o.policy);
+  if (o.q_stride < 1) return fail(PF_ERR_ARG, "q_stride %d < 1", o.q_stride);
+  if (o.head_lo < 0 || o.head_hi > cf.heads || o.head_lo >= o.head_hi)
+    return fail(PF_ERR_ARG, "head range [%d, %d) not inside [0, %d)", o.head_lo, o.head_hi, cf.heads);
+  if (o.heads_total < 0) return fail(PF_ERR_ARG, "heads_total %d < 0", o.heads_total);
+  const bool scored = o.policy == PF_ROUTE_SCORE || o.policy == PF_ROUTE_SCORES_ONLY;
+  if (scored && (s = check_ptr(Q, "Q")) != PF_OK) return s;
+  if (o.policy == PF_ROUTE_GIVEN) {
+    if (o.scores_in == nullptr) return fail(PF_ERR_ARG, "PF_ROUTE_GIVEN needs scores_in");
+    if (reinterpret_cast<uintptr_t>(o.scores_in) % 4 != 0) return fail(PF_ERR_ARG, "scores_in is not 4-byte aligned");
+  }
+  if (o.policy == PF_ROUTE_SCORES_ONLY && scores_out == nullptr)
+    return fail(PF_ERR_ARG, "PF_ROUTE_SCORES_ONLY needs scores_out");
+  Layer& Ly = c->L[layer];
+  const bool stores = o.policy != PF_ROUTE_SCORES_ONLY;
+  if (Ly.mid_count == 0 || (stores && cf.n_top == 0)) {
+    if (stores) {
+      Ly.sel_valid = true;
+      Ly.n_sel = 0;
+    }
     return PF_OK;
   }
   pf::SelectArgs a;
@@ -522,19 +547,48 @@ pf_status pf_select_mid(pf_cache* c, int layer, const void* Q, int32_t* sel_out,
   a.count = Ly.mid_count;
   a.chunk_rows = g.chunk_rows;
   a.chunks_per_block = 1;   // one partial per block: the dot product with its mean key
-  a.score_scale = static_cast<float>(1.0 / (static_cast<double>(g.n) * cf.heads * std::sqrt(128.0)));
+  const int rows = (g.n + o.q_stride - 1) / o.q_stride;
+  const int heads_norm = o.heads_total > 0 ? o.heads_total : o.head_hi - o.head_lo;
+  a.score_scale = static_cast<float>(1.0 / (static_cast<double>(rows) * heads_norm * std::sqrt(128.0)));
   a.partial = Ly.partial;
+  a.partial_ld = g.slots;
   a.scores = Ly.scores;
   a.ticket = Ly.ticket;
   a.n_top = cf.n_top;
   a.sel_slots = Ly.sel;
   a.sel_out = sel_out;
   a.scores_out = scores_out;
-  cudaError_t e = pf::launch_select(a, static_cast<cudaStream_t>(stream));
+  a.q_stride = o.q_stride;
+  a.d_lo = o.head_lo * 128;
+  a.d_hi = o.head_hi * 128;
+  a.topk = stores ? 1 : 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  switch (o.policy) {
+    case PF_ROUTE_SCORE:
+    case PF_ROUTE_SCORES_ONLY:
+      e = pf::launch_select(a, st);
+      break;
+    case PF_ROUTE_GIVEN:
+      a.partial = const_cast<float*>(o.scores_in);
+      a.partial_ld = Ly.mid_count;
+      a.score_scale = 1.f;
+      e = pf::launch_topk_given(a, st);
+      break;
+    default:
+      e = pf::launch_select_fifo(a, st);
+      break;
+  }
   if (e != cudaSuccess) return cuda_fail(e, "select launch");
-  Ly.sel_valid = true;
-  Ly.n_sel = cf.n_top < Ly.mid_count ? cf.n_top : Ly.mid_count;
+  if (stores) {
+    Ly.sel_valid = true;
+    Ly.n_sel = cf.n_top < Ly.mid_count ? cf.n_top : Ly.mid_count;
+  }
   return PF_OK;
+}
+
+pf_status pf_select_mid(pf_cache* c, int layer, const void* Q, int32_t* sel_out, float* scores_out, void* stream) {
+  return pf_select_mid_ex(c, layer, Q, nullptr, sel_out, scores_out, stream);
 }
 
 pf_status pf_rope_shift(pf_cache* c, int layer, unsigned parts, int delta, void* stream) {

@@ -63,9 +63,19 @@ struct SelectArgs {
   int32_t* sel_slots;   // [B, n_top] pool slots, ascending age
   int32_t* sel_out;     // optional [B, k] ages
   float* scores_out;    // optional [B, count]
+  int q_stride;         // query rows 0, q_stride, 2 q_stride, ... are pooled
+  int d_lo, d_hi;       // elements [d_lo, d_hi) of a token's H * D vector enter the score
+  int topk;             // 0: write the scores only (no selection)
+  int partial_ld;       // per-batch-item length of `partial`
 };
 
+// qpool + scoring (+ top-k unless a.topk == 0).
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
+// Top-k of given scores: a.partial holds [B, partial_ld] scores by age
+// (chunks_per_block = 1, score_scale = 1).
+cudaError_t launch_topk_given(const SelectArgs& a, cudaStream_t st);
+// The min(n_top, count) most recent live blocks.
+cudaError_t launch_select_fifo(const SelectArgs& a, cudaStream_t st);
 
 // kbar[b, slot] = mean of the block's n_c keys, slots [slot0, slot0 + nslots).
 cudaError_t launch_kmean(const void* pool_k, float* kbar, int B, int slots, int n_c, int HD, int slot0, int nslots,

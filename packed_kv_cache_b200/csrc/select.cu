@@ -73,14 +73,16 @@ __global__ void __launch_bounds__(kQcThreads, 2) qpool_kernel(const SelectArgs a
   const int phase = t >> 1;
   const uint4* Q = static_cast<const uint4*>(a.Q) + static_cast<long long>(b) * a.n * G + g;
   float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  // pooled rows: 0, q_stride, 2 q_stride, ... (nr of them)
+  const int nr = (a.n + a.q_stride - 1) / a.q_stride;
   if (g < G) {
-    const long long stride = static_cast<long long>(kQcPhases) * G;
-    const uint4* q = Q + static_cast<long long>(phase) * G;
-    for (int r = phase; r < a.n; r += kQcLoads * kQcPhases, q += kQcLoads * stride) {
+    const long long stride = static_cast<long long>(kQcPhases) * a.q_stride * G;
+    const uint4* q = Q + static_cast<long long>(phase) * a.q_stride * G;
+    for (int r = phase; r < nr; r += kQcLoads * kQcPhases, q += kQcLoads * stride) {
       uint4 w[kQcLoads];
 #pragma unroll
       for (int k = 0; k < kQcLoads; ++k)
-        w[k] = r + k * kQcPhases < a.n ? __ldg(q + k * stride) : make_uint4(0u, 0u, 0u, 0u);
+        w[k] = r + k * kQcPhases < nr ? __ldg(q + k * stride) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
       for (int k = 0; k < kQcLoads; ++k) acc_bf16x8(acc, w[k]);
     }
@@ -144,13 +146,17 @@ __device__ void select_tail(const SelectArgs& a, int b, uint32_t* keys) {
   const int t = threadIdx.x;
   const int count = a.count;
   for (int q = t; q < count; q += kThreads) {
-    const float* pp = a.partial + (static_cast<long long>(b) * a.slots + q) * a.chunks_per_block;
+    const float* pp = a.partial + static_cast<long long>(b) * a.partial_ld + static_cast<long long>(q) * a.chunks_per_block;
     float s = 0.f;
     for (int k = 0; k < a.chunks_per_block; ++k) s += __ldcg(pp + k);
     s *= a.score_scale;
     keys[q] = order_key(s);
     a.scores[static_cast<long long>(b) * a.slots + q] = s;
     if (a.scores_out) a.scores_out[static_cast<long long>(b) * count + q] = s;
+  }
+  if (!a.topk) {   // scores only
+    if (t == 0) a.ticket[b] = 0u;
+    return;
   }
   const int k_sel = min(a.n_top, count);
   if (t == 0) {
@@ -266,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 5) score_kernel(const SelectArgs a) 
   if (t == 0) {
     float s = 0.f;
     for (int k = 0; k < kThreads / 32; ++k) s += red[k];
-    a.partial[(static_cast<long long>(b) * a.slots + p) * a.chunks_per_block + c] = s;
+    a.partial[static_cast<long long>(b) * a.partial_ld + static_cast<long long>(p) * a.chunks_per_block + c] = s;
     __threadfence();
     const unsigned total = static_cast<unsigned>(a.count * a.chunks_per_block);
     is_last = (atomicAdd(&a.ticket[b], 1u) == total - 1u) ? 1u : 0u;
@@ -293,11 +299,12 @@ __global__ void __launch_bounds__(kThreads) score_mean_kernel(const SelectArgs a
   if (p < a.count) {
     const int slot = (a.head + p) % a.slots;
     const float4* q = reinterpret_cast<const float4*>(qs);
+    // elements [d_lo, d_hi) of the mean key: the heads that enter the score
     const float4* k = reinterpret_cast<const float4*>(a.kbar + (static_cast<long long>(b) * a.slots + slot) * a.HD);
-    const int nv = a.HD / 4;
+    const int nv = a.d_hi / 4;
     float acc = 0.f;
     // eight 16-byte loads of the mean key in flight per lane
-    for (int i0 = lane; i0 < nv; i0 += 32 * 8) {
+    for (int i0 = a.d_lo / 4 + lane; i0 < nv; i0 += 32 * 8) {
       float4 y[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
@@ -315,7 +322,7 @@ __global__ void __launch_bounds__(kThreads) score_mean_kernel(const SelectArgs a
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) a.partial[static_cast<long long>(b) * a.slots + p] = acc;
+    if (lane == 0) a.partial[static_cast<long long>(b) * a.partial_ld + p] = acc;
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -364,6 +371,23 @@ __global__ void __launch_bounds__(kThreads) kmean_kernel(const void* pool_k, flo
 
 }  // namespace
 
+// Top-k of given scores, one CTA per batch item (a.partial = the scores).
+__global__ void __launch_bounds__(kThreads) topk_given_kernel(const SelectArgs a) {
+  extern __shared__ float smem[];
+  select_tail(a, blockIdx.x, reinterpret_cast<uint32_t*>(smem));
+}
+
+// The k = min(n_top, count) most recent live blocks, ascending age.
+__global__ void fifo_kernel(const SelectArgs a) {
+  const int b = blockIdx.x;
+  const int k = min(a.n_top, a.count);
+  for (int i = threadIdx.x; i < k; i += blockDim.x) {
+    const int q = a.count - k + i;
+    a.sel_slots[static_cast<long long>(b) * a.n_top + i] = (a.head + q) % a.slots;
+    if (a.sel_out) a.sel_out[static_cast<long long>(b) * k + i] = q;
+  }
+}
+
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
   if (a.count <= 0) return cudaSuccess;
   dim3 g1((a.HD / 8 + 1) / 2, a.B);
@@ -388,6 +412,24 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
   }
   dim3 g2(a.count * a.chunks_per_block, a.B);
   score_kernel<<<g2, kThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_given(const SelectArgs& a, cudaStream_t st) {
+  if (a.count <= 0) return cudaSuccess;
+  const size_t smem = static_cast<size_t>(a.count) * 4;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(topk_given_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  topk_given_kernel<<<a.B, kThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_fifo(const SelectArgs& a, cudaStream_t st) {
+  if (a.count <= 0) return cudaSuccess;
+  fifo_kernel<<<a.B, 128, 0, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -510,6 +552,11 @@ extern "C" pf_status pf_select_mid_static(const void* Q, int batch, int n, int h
   a.sel_slots = sc->sel_slots;
   a.sel_out = sel_out;
   a.scores_out = scores_out;
+  a.q_stride = 1;
+  a.d_lo = 0;
+  a.d_hi = HD;
+  a.topk = 1;
+  a.partial_ld = pool_slots * a.chunks_per_block;
   e = launch_select(a, st);
   if (e != cudaSuccess)
     return static_cast<pf_status>(report_error(PF_ERR_CUDA, "select launch: %s", cudaGetErrorString(e)));

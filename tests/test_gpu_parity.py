@@ -183,6 +183,117 @@ def test_selection_ties_go_to_older_blocks(pf):
     assert sel.cpu().tolist() == [[0, 1, 2, 3]] * wl.batch
 
 
+# ------------------------------------------------- selection routing options
+
+def _sel_inputs(name):
+    wl = _wl(name)
+    d = synth.make_layer(wl, seed_for(name), device="cpu", with_values=False)
+    for k in ("mid_V", "sink_V", "recent_V"):
+        d[k] = torch.zeros_like(d[k.replace("V", "K")])
+    d["V_cur"] = torch.zeros_like(d["K_cur"])
+    return wl, d
+
+
+@pytest.mark.parametrize("name,q_stride,heads", [("ragged_a", 4, None), ("ragged_c", 4, (0, 1)),
+                                                 ("ragged_c", 7, (1, 3)), ("layer", 4, (0, 6)),
+                                                 ("stress16", 1, (0, 6)), ("stress16", 7, (6, 12))])
+def test_selection_subsampled_queries_and_head_range(pf, name, q_stride, heads):
+    # the speed variant: every q_stride-th query row, a head range
+    wl, d = _sel_inputs(name)
+    cache = build_cache(pf, wl, d)
+    B, P = wl.batch, wl.pool_blocks
+    k = min(wl.n_top, P)
+    sel = torch.full((B, k), -1, dtype=torch.int32, device="cuda")
+    sc = torch.zeros((B, P), dtype=torch.float32, device="cuda")
+    cache.select_mid_ex(0, d["Q"].cuda(), q_stride=q_stride, heads=heads, sel_out=sel, scores_out=sc)
+    torch.cuda.synchronize()
+    S_ref = oracle.select_scores(d["Q"], d["mid_K"], q_stride=q_stride, heads=heads)
+    assert np.all(oracle.selection_margin(S_ref, wl.n_top) >= 1e-3)
+    assert np.array_equal(sel.cpu().numpy(), oracle.select_topk(S_ref, wl.n_top))
+    scale = np.abs(S_ref).max(axis=1, keepdims=True)
+    assert np.max(np.abs(sc.cpu().numpy() - S_ref) / scale) < 1e-4
+    assert cache.info(0)["selection_valid"] == 1
+
+
+def test_head_shard_scores_sum_then_given_top_k(pf):
+    # two disjoint head ranges divided by the total head count (what two GPUs
+    # holding six heads each would compute), summed, then the top-k of the
+    # sum: the same selection and the same attention as the all-head call
+    wl, d = _layer("ragged_b")
+    cache = build_cache(pf, wl, d)
+    B, P, H = wl.batch, wl.pool_blocks, wl.heads
+    k = min(wl.n_top, P)
+    Q, Kc, Vc = d["Q"].cuda(), d["K_cur"].cuda(), d["V_cur"].cuda()
+    sel_full = torch.full((B, k), -1, dtype=torch.int32, device="cuda")
+    sc_full = torch.zeros((B, P), dtype=torch.float32, device="cuda")
+    cache.select_mid(0, Q, sel_full, sc_full)
+    O_full = cache.attend(0, Q, Kc, Vc)
+    half = H // 2
+    parts = []
+    for lo, hi in ((0, half), (half, H)):
+        sc = torch.zeros((B, P), dtype=torch.float32, device="cuda")
+        cache.select_mid_ex(0, Q, policy=pf.ROUTE_SCORES_ONLY, heads=(lo, hi), heads_total=H, scores_out=sc)
+        parts.append(sc)
+    summed = parts[0] + parts[1]
+    torch.cuda.synchronize()
+    scale = sc_full.abs().max().item()
+    assert (summed - sc_full).abs().max().item() <= 1e-5 * scale
+    S_ref = oracle.select_scores(d["Q"], d["mid_K"])
+    half_ref = oracle.select_scores(d["Q"], d["mid_K"], heads=(0, half), heads_norm=H)
+    assert np.max(np.abs(parts[0].cpu().numpy() - half_ref)) <= 1e-4 * np.abs(S_ref).max()
+    sel_g = torch.full((B, k), -1, dtype=torch.int32, device="cuda")
+    cache.select_mid_ex(0, policy=pf.ROUTE_GIVEN, scores_in=summed.contiguous(), sel_out=sel_g)
+    O_g = cache.attend(0, Q, Kc, Vc)
+    torch.cuda.synchronize()
+    assert torch.equal(sel_g, sel_full)
+    assert torch.equal(O_g, O_full)
+
+
+@pytest.mark.parametrize("name", ["ragged_b", "ragged_c"])
+def test_random_and_fifo_routing_then_attention(pf, name):
+    # the pages' routing baselines: random blocks (random scores passed in)
+    # and FIFO (the newest blocks); attention runs over what was routed
+    wl, d = _layer(name)
+    cache = build_cache(pf, wl, d)
+    B, P = wl.batch, wl.pool_blocks
+    k = min(wl.n_top, P)
+    Q, Kc, Vc = d["Q"].cuda(), d["K_cur"].cuda(), d["V_cur"].cuda()
+    rng = np.random.default_rng(3)
+    rand = np.stack([rng.permutation(P) for _ in range(B)]).astype(np.float32)   # distinct scores
+    sel = torch.full((B, k), -1, dtype=torch.int32, device="cuda")
+    cache.select_mid_ex(0, policy=pf.ROUTE_GIVEN, scores_in=torch.from_numpy(rand).cuda(), sel_out=sel)
+    O = cache.attend(0, Q, Kc, Vc)
+    torch.cuda.synchronize()
+    sel_ref = oracle.select_topk(rand, wl.n_top)
+    assert np.array_equal(sel.cpu().numpy(), sel_ref)
+    O_ref, _ = oracle.attend(d["Q"], oracle_context(wl, d, sel_ref))
+    assert_attention_close(O.cpu(), O_ref, f"{name} random routing")
+    sel_f = torch.full((B, k), -1, dtype=torch.int32, device="cuda")
+    cache.select_mid_ex(0, policy=pf.ROUTE_FIFO, sel_out=sel_f)
+    O = cache.attend(0, Q, Kc, Vc)
+    torch.cuda.synchronize()
+    fifo = np.stack([oracle.select_fifo(P, wl.n_top)] * B)
+    assert np.array_equal(sel_f.cpu().numpy(), fifo)
+    O_ref, _ = oracle.attend(d["Q"], oracle_context(wl, d, fifo))
+    assert_attention_close(O.cpu(), O_ref, f"{name} FIFO routing")
+
+
+def test_select_ex_rejects_bad_options(pf):
+    wl, d = _sel_inputs("ragged_a")
+    cache = build_cache(pf, wl, d)
+    Q = d["Q"].cuda()
+    sc = torch.zeros((wl.batch, wl.pool_blocks), dtype=torch.float32, device="cuda")
+    bad = [dict(policy=9), dict(q_stride=0), dict(heads=(1, 1)), dict(heads=(0, wl.heads + 1)),
+           dict(heads=(-1, 1)), dict(heads_total=-2), dict(policy=pf.ROUTE_GIVEN),
+           dict(policy=pf.ROUTE_SCORES_ONLY)]
+    for kw in bad:
+        with pytest.raises(pf.PFError) as e:
+            cache.select_mid_ex(0, Q, **kw)
+        assert e.value.status_name == "PF_ERR_ARG", kw
+    with pytest.raises(pf.PFError):
+        cache.select_mid_ex(0, None, scores_out=sc)      # scoring needs Q
+
+
 # ------------------------------------------------------------------ attention
 
 def _attend_and_compare(pf, wl, d, rows=None, via_append=False, lse_check=True):

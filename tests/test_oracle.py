@@ -201,6 +201,41 @@ def test_selection_small_pool_and_ties():
     assert oracle.selection_margin(np.array([[3.0, 1.0, 2.0]]), 1)[0] == pytest.approx(1 / 3)
 
 
+def test_subsampled_half_head_scores_equal_bruteforce_on_the_slices():
+    # the selection's speed variant (digest, limitations paragraph): every
+    # q_stride-th query and a head range; pinned by the token-level double
+    # sum over exactly those queries and heads
+    wl = synth.WORKLOADS["ragged_c"]
+    d = synth.make_layer(wl.replace(pool_blocks=5, planted=2), 11)
+    a = oracle.select_scores(d["Q"], d["mid_K"], q_stride=3, heads=(1, 3))
+    b = oracle.select_scores_bruteforce(d["Q"][:, ::3, 1:3], d["mid_K"][:, :, :, 1:3])
+    assert np.max(np.abs(a - b) / np.max(np.abs(b))) < 1e-10
+    # one head, stride larger than the block: only query row 0
+    c = oracle.select_scores(d["Q"], d["mid_K"], q_stride=10_000, heads=(2, 3))
+    e = oracle.select_scores_bruteforce(d["Q"][:, :1, 2:3], d["mid_K"][:, :, :, 2:3])
+    assert np.max(np.abs(c - e) / np.max(np.abs(e))) < 1e-10
+
+
+def test_head_shard_scores_add_up_to_the_full_score():
+    # disjoint head ranges divided by the total head count sum to the score
+    wl = synth.WORKLOADS["ragged_c"]
+    d = synth.make_layer(wl.replace(pool_blocks=6, planted=2), 12)
+    H = d["Q"].shape[2]
+    full = oracle.select_scores(d["Q"], d["mid_K"])
+    parts = sum(oracle.select_scores(d["Q"], d["mid_K"], heads=(lo, lo + 1), heads_norm=H) for lo in range(H))
+    assert np.max(np.abs(parts - full)) < 1e-14 * max(1.0, np.max(np.abs(full))) * 10
+    assert np.array_equal(oracle.select_topk(parts, 2), oracle.select_topk(full, 2))
+
+
+def test_fifo_routing_is_top_k_of_age():
+    # FIFO keeps the newest blocks: the same as ranking by age
+    for count, k in [(40, 16), (5, 16), (16, 16), (1, 1), (7, 0)]:
+        f = oracle.select_fifo(count, k)
+        assert f.tolist() == (oracle.select_topk(np.arange(count, dtype=np.float64)[None], k)[0].tolist()
+                              if k else [])
+        assert len(f) == min(k, count)
+
+
 # ---------------------------------------------------------------- attention
 
 def _rand(shape, seed):
