@@ -474,8 +474,9 @@ def run_suite(args):
     iters = max(args.steps, 5)
     out = []
 
-    def build(wl, d):
-        cache = pf.PackedKVCache(pf.config_for(wl, layers=1), device=dev)
+    def build(wl, d, sink_rope_in_attention=False):
+        cache = pf.PackedKVCache(pf.config_for(wl, layers=1, sink_rope_in_attention=sink_rope_in_attention),
+                                 device=dev)
         for s_ in range(wl.sink_blocks):
             cache.append_block(0, d["sink_K"][:, s_].contiguous(), d["sink_V"][:, s_].contiguous())
         if wl.pool_blocks:
@@ -542,6 +543,17 @@ def run_suite(args):
         Lk = cache.info(0)["context_tokens"]
         ms = _timed(lambda: cache.attend(0, d["Q"], d["K_cur"], d["V_cur"], O), iters, flush, stream)
         out.append(line("attend", f"layer (Lk {Lk})", ms, "tensor", attention_flops(B, H, n, Lk, D), None))
+        cache.poll_device_error()
+        del cache
+        torch.cuda.empty_cache()
+        # the sink's RoPE shift applied inside attention (sink K tiles rotated
+        # in shared memory); the in-place shift pass disappears from the step
+        cache = build(wl, d, sink_rope_in_attention=True)
+        cache.rope_shift(0, pf.PART_SINK, 4)
+        cache.select_mid(0, d["Q"])
+        ms = _timed(lambda: cache.attend(0, d["Q"], d["K_cur"], d["V_cur"], O), iters, flush, stream)
+        out.append(line("attend, sink RoPE shift applied in attention", f"layer (Lk {Lk})", ms, "tensor",
+                        attention_flops(B, H, n, Lk, D), None))
         cache.poll_device_error()
         del cache
         torch.cuda.empty_cache()

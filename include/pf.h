@@ -68,6 +68,10 @@ typedef struct pf_config {
   int n_top;         /* N_top: mid blocks routed into attention (16) */
   int rope_split[3]; /* rotary dims per axis (temporal, height, width) = 44, 42, 42 */
   float rope_base;   /* rotary base (10000) */
+  int sink_rope_in_attention; /* 0: pf_rope_shift rotates the stored sink keys in place;
+                                 1: it records the shift and pf_attend rotates the sink's
+                                 key tiles as they are loaded (the stored keys stay as
+                                 appended; see pf_rope_shift) */
 } pf_config;
 
 typedef struct pf_cache pf_cache;
@@ -237,6 +241,15 @@ pf_status pf_select_mid_ex(pf_cache* cache, int layer, const void* Q, const pf_s
  * One kernel launch per layer.
  */
 pf_status pf_rope_shift(pf_cache* cache, int layer, unsigned parts, int delta, void* stream);
+/*
+ * With sink_rope_in_attention = 1 the sink part of a shift launches
+ * nothing: the layer's total shift (pf_layer_info.total_shift) is applied
+ * by pf_attend to the sink's key tiles in shared memory, between their load
+ * and the QK^T MMA, with the same float32 rotation and bf16 rounding (one
+ * rounding for the whole accumulated shift).  The sink must then be full
+ * before its first shift (PF_ERR_STATE otherwise), since every stored sink
+ * key is rotated by the same total.
+ */
 
 /*
  * Attention of the current block's queries over the bounded context

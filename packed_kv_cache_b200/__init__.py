@@ -47,7 +47,8 @@ class Config(ctypes.Structure):
                 ("head_dim", ctypes.c_int), ("block_frames", ctypes.c_int), ("h", ctypes.c_int),
                 ("w", ctypes.c_int), ("sink_blocks", ctypes.c_int), ("recent_blocks", ctypes.c_int),
                 ("mid_capacity", ctypes.c_int), ("n_top", ctypes.c_int),
-                ("rope_split", ctypes.c_int * 3), ("rope_base", ctypes.c_float)]
+                ("rope_split", ctypes.c_int * 3), ("rope_base", ctypes.c_float),
+                ("sink_rope_in_attention", ctypes.c_int)]
 
 
 class SelectOpts(ctypes.Structure):
@@ -130,9 +131,10 @@ def _stream(stream) -> int | None:
     return int(stream)
 
 
-def config_for(wl, layers: int | None = None) -> Config:
+def config_for(wl, layers: int | None = None, sink_rope_in_attention: bool = False) -> Config:
     """A pf_config for a workload description (``synth.Workload`` or alike)."""
     c = Config()
+    c.sink_rope_in_attention = 1 if sink_rope_in_attention else 0
     c.layers = layers if layers is not None else getattr(wl, "layers", 1)
     c.batch, c.heads, c.head_dim = wl.batch, wl.heads, wl.head_dim
     c.block_frames, c.h, c.w = wl.block_frames, wl.h, wl.w

@@ -20,6 +20,8 @@
 //   warp 0      TMA producer: Q, then K and V tiles through rings
 //   warp 1      MMA issuer (one thread): S_t = Q_t K^T and O_t += P_t V
 //   warp 2      tensor-memory allocator
+//   warps 2-3   when the sink's RoPE shift is applied here: rotate the sink
+//               rows of each K tile in shared memory after TMA lands it
 //   warps 4-7   softmax of query tile 0 (one thread per query row)
 //   warps 8-11  softmax of query tile 1
 // Tensor memory (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each;
@@ -56,6 +58,7 @@ constexpr uint32_t kTileBytes = kBN * kHeadDim * 2;   // 32 KB
 constexpr uint32_t kHalfBytes = kTileBytes / 2;       // 64 dims x 128 rows
 constexpr uint32_t kSubBytes = kSub * 128;            // one sub-box, one 64-dim half
 constexpr float kRescaleThreshold = 8.0f;
+constexpr int kRotThreads = 64;   // warps 2-3
 // Before S_t of the next tile is written over P_t, wait until the P_t V MMA
 // that reads P_t has completed.  Off by default: tcgen05.mma operations
 // issued by one thread execute in issue order.
@@ -87,6 +90,7 @@ static_assert(kSmemBytes <= 232448, "shared memory");
 struct Bars {
   uint64_t q_full;
   uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t k_ready[kKStages];   // K tile rotated (only used when rotate_sink)
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2], o_final[2];
   uint64_t drain;
@@ -267,6 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(&bars.k_full[s], 1);
       mbar_init(&bars.k_empty[s], 1);
+      mbar_init(&bars.k_ready[s], kRotThreads);
     }
     for (int s = 0; s < kVStages; ++s) {
       mbar_init(&bars.v_full[s], 1);
@@ -373,8 +378,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
           mma_ts(tO[t], tS[t] + kk * 8, sdesc_sw128(va + kk * 2048, kHalfBytes, 1024), idesc_pv,
                  (!first || kk > 0) ? 1u : 0u);
       };
+      uint64_t* k_avail = p.rotate_sink ? bars.k_ready : bars.k_full;
       auto wait_k = [&](int g, unsigned site) {
-        return mbar_wait_bounded(&bars.k_full[g % kKStages], (g / kKStages) & 1, abort_flag, p.err,
+        return mbar_wait_bounded(&k_avail[g % kKStages], (g / kKStages) & 1, abort_flag, p.err,
                                  kDevErrTimeoutBase | site, lim);
       };
       int kg = 0, vg = 0, drains = 0;
@@ -462,6 +468,55 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
       if (!ok) {
         // make sure nothing issued is still running before the memory goes away
         mbar_wait_bounded(&bars.o_final[0], 0, nullptr, nullptr, 0, lim / 4 + 1);
+      }
+    }
+  } else if (warp == 2 || warp == 3) {
+    if (p.rotate_sink) {
+      // ------------------------------------------------ sink-key rotator
+      // PackForcing (arXiv), "Incremental RoPE adjustment": the sink keys'
+      // temporal pairs times e^{i theta_k total_shift}, applied to the K tile
+      // in shared memory (dims 0-63 half, 128-byte swizzle: 16-byte chunk c
+      // of row r sits at chunk c ^ (r & 7)); the MMA issuer waits for k_ready.
+      // thread rt owns 16-byte word c = rt % 8 (pairs 4c .. 4c+3, their
+      // cosines and sines kept in registers) of rows rt / 8 + 8 m
+      const int rt = threadIdx.x - 64;
+      const int c = rt & 7, r0 = rt >> 3;
+      const int sink_tiles = (p.sb_sink + 3) / 4;
+      const bool active = c * 4 < p.sink_rope.pairs;
+      float cs[4], sn[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        cs[q] = p.sink_rope.c[(c * 4 + q) & 31];
+        sn[q] = p.sink_rope.s[(c * 4 + q) & 31];
+      }
+      bool ok = true;
+      int kg = 0;
+      for (int j = un.j0; ok && j < un.j1; ++j, ++kg) {
+        const int st = kg % kKStages;
+        ok = mbar_wait_bounded(&bars.k_full[st], (kg / kKStages) & 1, abort_flag, p.err, kDevErrTimeoutBase | 14u,
+                               lim);
+        if (!ok) break;
+        if (j < sink_tiles && active) {
+          const int nsb = min(4, p.sb_sink - 4 * j);   // the tile's first nsb sub-boxes are sink rows
+          uint8_t* tile = smem + kOffK + st * kTileBytes;
+          for (int i = 0; i < nsb; ++i) {
+            uint4 w[kSub / 8];
+            uint4* ptr[kSub / 8];
+#pragma unroll
+            for (int m = 0; m < kSub / 8; ++m) {
+              const int rr = r0 + 8 * m;
+              ptr[m] = reinterpret_cast<uint4*>(tile + i * kSubBytes + rr * 128 + ((c ^ (rr & 7)) << 4));
+              w[m] = *ptr[m];
+            }
+#pragma unroll
+            for (int m = 0; m < kSub / 8; ++m) {
+              rope_rotate_word_cs(w[m], c, p.sink_rope.pairs, cs, sn);
+              *ptr[m] = w[m];
+            }
+          }
+          fence_proxy_async_smem();
+        }
+        mbar_arrive(&bars.k_ready[st]);
       }
     }
   } else if (warp >= 4) {
@@ -607,6 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
   tc_fence_before();
   __syncthreads();
   if (warp == 2) {
+    __syncwarp();   // the allocating warp may have run the rotator loop
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

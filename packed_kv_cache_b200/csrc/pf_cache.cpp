@@ -72,6 +72,8 @@ pf_status check_config(const pf_config* c) {
     return fail(PF_ERR_UNSUPPORTED, "rope_split must be three even sizes summing to head_dim");
   if (s[0] > 64) return fail(PF_ERR_UNSUPPORTED, "at most 64 temporal rotary dims (got %d)", s[0]);
   if (!(c->rope_base > 1.0f)) return fail(PF_ERR_ARG, "rope_base must be > 1");
+  if (c->sink_rope_in_attention != 0 && c->sink_rope_in_attention != 1)
+    return fail(PF_ERR_ARG, "sink_rope_in_attention must be 0 or 1");
   const long long n = 1LL * c->block_frames * c->h * c->w;
   if (n > (1 << 24)) return fail(PF_ERR_CAPACITY, "block of %lld tokens is too large", n);
   const long long n_c = 1LL * (c->block_frames / 2) * (c->h / 4) * (c->w / 4);
@@ -620,9 +622,15 @@ pf_status pf_rope_shift(pf_cache* c, int layer, unsigned parts, int delta, void*
   const int l0 = layer < 0 ? 0 : layer, l1 = layer < 0 ? cf.layers : layer + 1;
   const long long H = cf.heads;
   const size_t rowb = static_cast<size_t>(g.HD) * 2;
+  const bool sink_lazy = cf.sink_rope_in_attention != 0;
+  if ((parts & PF_PART_SINK) && sink_lazy)
+    for (int l = l0; l < l1; ++l)
+      if (c->L[l].sink_filled < cf.sink_blocks)
+        return fail(PF_ERR_STATE, "layer %d: the sink shift is applied in attention and needs a full sink (%d of %d "
+                    "blocks)", l, c->L[l].sink_filled, cf.sink_blocks);
   for (int l = l0; l < l1; ++l) {
     Layer& Ly = c->L[l];
-    if (parts & PF_PART_SINK) {
+    if ((parts & PF_PART_SINK) && !sink_lazy) {
       if (Ly.sink_filled == cf.sink_blocks) {
         rb.add(Ly.sink_k, 1LL * cf.batch * cf.sink_blocks * g.n * H);
       } else {
@@ -744,6 +752,18 @@ pf_status pf_attend(pf_cache* c, int layer, const void* Q, const void* K_cur, co
   p.part_o = c->part_o;
   p.part_ml = c->part_ml;
   p.tail_ticket = c->tail_ticket;
+  p.rotate_sink = (cf.sink_rope_in_attention && Ly.total_shift != 0 && sink_rows > 0) ? 1 : 0;
+  p.sink_rope.pairs = cf.rope_split[0] / 2;
+  for (int k = 0; k < 32; ++k) {
+    p.sink_rope.c[k] = 1.f;
+    p.sink_rope.s[k] = 0.f;
+  }
+  for (int k = 0; k < p.sink_rope.pairs; ++k) {
+    const double theta = std::pow(static_cast<double>(cf.rope_base), -2.0 * k / cf.rope_split[0]);
+    const double ang = theta * static_cast<double>(Ly.total_shift);
+    p.sink_rope.c[k] = static_cast<float>(std::cos(ang));
+    p.sink_rope.s[k] = static_cast<float>(std::sin(ang));
+  }
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
   p.err = c->err;
   p.timeout_cycles = c->timeout_cycles;

@@ -29,6 +29,42 @@ struct RopeTable {
   float s[32];
 };
 
+#ifdef __CUDACC__
+// Rotate the rotary pairs held in 16-byte word `word` (bf16 pairs 4 word ..
+// 4 word + 3) of a key vector: (re, im) -> (re c - im s, re s + im c) in
+// float32, rounded to bf16 (nearest even); cs / sn hold the four pairs'
+// cosines and sines.  Pairs at or past `pairs` stay.  Shared by the
+// in-place shift and the shift applied inside attention, so both round
+// identically.
+__device__ __forceinline__ void rope_rotate_word_cs(uint4& w, int word, int pairs, const float* cs,
+                                                    const float* sn) {
+  uint32_t v[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (word * 4 + q < pairs) {
+      const float re = __uint_as_float(v[q] << 16), im = __uint_as_float(v[q] & 0xffff0000u);
+      const float nre = re * cs[q] - im * sn[q];
+      const float nim = re * sn[q] + im * cs[q];
+      uint32_t r;
+      asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(nim), "f"(nre));
+      v[q] = r;
+    }
+  }
+  w = make_uint4(v[0], v[1], v[2], v[3]);
+}
+
+__device__ __forceinline__ void rope_rotate_word(uint4& w, int word, const RopeTable& t) {
+  float cs[4], sn[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int pair = (word * 4 + q) & 31;
+    cs[q] = t.c[pair];
+    sn[q] = t.s[pair];
+  }
+  rope_rotate_word_cs(w, word, t.pairs, cs, sn);
+}
+#endif
+
 cudaError_t launch_rope_shift(const RowRuns& runs, const RopeTable& tab, cudaStream_t st);
 // The same rotation of float32 128-dim vectors (cached mean keys); runs count vectors.
 cudaError_t launch_rope_shift_f32(const RowRuns& runs, const RopeTable& tab, cudaStream_t st);
@@ -108,6 +144,8 @@ struct AttendParams {
   float* part_o;        // [tails * tail_chunks, 128, 128] unnormalised partial outputs
   float* part_ml;       // [tails * tail_chunks, 2, 128] partial row max / row sum
   unsigned* tail_ticket;  // [tails], zero on entry, left zero on exit
+  int rotate_sink;      // 1: rotate the sink keys' temporal pairs by sink_rope as they are loaded
+  RopeTable sink_rope;  // e^{i theta_k total_shift}
   float scale_log2;     // log2(e) / sqrt(D)
   unsigned* err;
   long long timeout_cycles;

@@ -23,24 +23,6 @@ namespace pf {
 
 namespace {
 
-__device__ __forceinline__ void rotate_word(uint4& w, int word, const RopeTable& t) {
-  uint32_t v[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int pair = word * 4 + q;
-    if (pair < t.pairs) {
-      __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&v[q]);
-      const float re = __low2float(x), im = __high2float(x);
-      const float c = t.c[pair], s = t.s[pair];
-      const float nre = re * c - im * s;
-      const float nim = re * s + im * c;
-      __nv_bfloat162 y = __floats2bfloat162_rn(nre, nim);
-      v[q] = *reinterpret_cast<uint32_t*>(&y);
-    }
-  }
-  w = make_uint4(v[0], v[1], v[2], v[3]);
-}
-
 template <int NW>
 __global__ void __launch_bounds__(256) rope_shift_kernel(const RowRuns runs, const RopeTable tab) {
   const long long total = runs.start[runs.n];
@@ -65,7 +47,7 @@ __global__ void __launch_bounds__(256) rope_shift_kernel(const RowRuns runs, con
     for (int u = 0; u < 2; ++u) {
       if (ptr[u] != nullptr) {
 #pragma unroll
-        for (int k = 0; k < NW; ++k) rotate_word(w[u][k], k, tab);
+        for (int k = 0; k < NW; ++k) rope_rotate_word(w[u][k], k, tab);
 #pragma unroll
         for (int k = 0; k < NW; ++k) ptr[u][k] = w[u][k];
       }

@@ -32,9 +32,10 @@ def seed_for(name: str) -> int:
     return synth.nominal_seed(list(synth.WORKLOADS).index(name))
 
 
-def build_cache(pf, wl, d, via_append: bool = False, device="cuda"):
+def build_cache(pf, wl, d, via_append: bool = False, device="cuda", sink_rope_in_attention: bool = False):
     """A one-layer cache holding d's sink, mid pool and recent blocks."""
-    cache = pf.PackedKVCache(pf.config_for(wl, layers=1), device=device)
+    cache = pf.PackedKVCache(pf.config_for(wl, layers=1, sink_rope_in_attention=sink_rope_in_attention),
+                             device=device)
     dev = lambda t: t.to(device).contiguous()  # noqa: E731
     for s in range(wl.sink_blocks):
         cache.append_block(0, dev(d["sink_K"][:, s]), dev(d["sink_V"][:, s]))

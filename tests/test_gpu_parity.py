@@ -458,13 +458,16 @@ def test_state_machine_against_partition_model(pf):
 
 # ------------------------------------------------------------------ generation loop
 
-def test_generation_loop_against_oracle_model(pf):
+@pytest.mark.parametrize("fused", [False, True])
+def test_generation_loop_against_oracle_model(pf, fused):
     """select -> attend -> append -> shift over several blocks, with the
-    oracle keeping its own copy of every partition."""
+    oracle keeping its own copy of every partition.  fused: the sink shift
+    is applied inside attention (one rounding of the accumulated shift)."""
     wl = _wl("ragged_a").replace(mid_capacity=4, n_top=2, planted=0)
     B, n, nc, H, D, Bf = wl.batch, wl.n, wl.n_c, wl.heads, wl.head_dim, wl.block_frames
-    cache = pf.PackedKVCache(pf.config_for(wl, layers=1))
+    cache = pf.PackedKVCache(pf.config_for(wl, layers=1, sink_rope_in_attention=fused))
     sinkK, sinkV, mid, recent = [], [], [], []     # oracle's partitions (bf16-valued float64 / tensors)
+    total = 0                                      # accumulated sink shift (fused)
     for i in range(12):
         blk = synth.make_block(wl, 7000 + i)
         Q = synth.bf16_normal((B, n, H, D), 9000 + i)
@@ -480,7 +483,11 @@ def test_generation_loop_against_oracle_model(pf):
             if np.all(oracle.selection_margin(S_ref, wl.n_top) >= 1e-3):
                 assert np.array_equal(sel, oracle.select_topk(S_ref, wl.n_top))
         O = cache.attend(0, qd, blk["K"].cuda(), blk["V"].cuda()).cpu()
-        parts = [(torch.from_numpy(k), v) for k, v in zip(sinkK, sinkV)]
+        if fused and total:
+            parts = [(torch.from_numpy(oracle.round_bf16(oracle.rope_shift(k, total))), v)
+                     for k, v in zip(sinkK, sinkV)]
+        else:
+            parts = [(torch.from_numpy(k), v) for k, v in zip(sinkK, sinkV)]
         if mid:
             chosen = [list(range(len(mid)))] * B if sel is None else sel.tolist()
             for j in range(len(chosen[0])):
@@ -505,8 +512,55 @@ def test_generation_loop_against_oracle_model(pf):
                     assert ev == 1
         if ev:
             cache.rope_shift(0, pf.PART_SINK, ev * Bf)
-            sinkK = [oracle.round_bf16(oracle.rope_shift(k, ev * Bf)) for k in sinkK]
+            if fused:
+                total += ev * Bf
+            else:
+                sinkK = [oracle.round_bf16(oracle.rope_shift(k, ev * Bf)) for k in sinkK]
     assert cache.info(0)["total_shift"] == cache.info(0)["evicted"] * Bf
+
+
+@pytest.mark.parametrize("name", ["ragged_a", "ragged_c", "layer"])
+def test_sink_rope_in_attention_matches_oracle(pf, name):
+    # the sink's shift recorded by pf_rope_shift and applied by pf_attend to
+    # the sink's key tiles: the stored keys stay as appended; attention sees
+    # them rotated by the accumulated shift (rounded to bf16 once)
+    wl, d = _layer(name)
+    cache = build_cache(pf, wl, d, sink_rope_in_attention=True)
+    info = cache.info(0)
+    B, S, n, H, D = wl.batch, wl.sink_blocks, wl.n, wl.heads, wl.head_dim
+    d1, d2 = d["delta"], 3 * d["delta"] + 5
+    cache.rope_shift(0, pf.PART_SINK, d1)
+    cache.rope_shift(0, pf.PART_SINK, d2)
+    Q, Kc, Vc = d["Q"].cuda(), d["K_cur"].cuda(), d["V_cur"].cuda()
+    k = min(wl.n_top, wl.pool_blocks)
+    s = torch.zeros((B, k), dtype=torch.int32, device="cuda")
+    cache.select_mid(0, Q, s, None)
+    O = cache.attend(0, Q, Kc, Vc)
+    assert cache.poll_device_error() == 0
+    O = O.cpu()
+    assert cache.info(0)["total_shift"] == d1 + d2
+    stored = arena_view(cache, info["sink_k"], (B, S * n, H, D)).cpu()
+    assert torch.equal(stored, d["sink_K"].reshape(B, S * n, H, D))     # not rotated in place
+    rot = dict(d)
+    rot["sink_K"] = torch.from_numpy(oracle.round_bf16(oracle.rope_shift(d["sink_K"], d1 + d2)))
+    rows = _rows(wl.n) if wl.n > 1000 else None
+    O_ref, _ = oracle.attend(d["Q"], oracle_context(wl, rot, s.cpu().numpy()), rows=rows)
+    got = O if rows is None else O[:, rows]
+    assert_attention_close(got, O_ref, f"{name} sink rope in attention")
+
+
+def test_sink_rope_in_attention_needs_a_full_sink(pf):
+    wl = _wl("ragged_a")
+    cache = pf.PackedKVCache(pf.config_for(wl, layers=1, sink_rope_in_attention=True))
+    blk = synth.make_block(wl, 17)
+    cache.append_block(0, blk["K"].cuda(), blk["V"].cuda())   # 1 of 2 sink blocks
+    with pytest.raises(pf.PFError) as e:
+        cache.rope_shift(0, pf.PART_SINK, 4)
+    assert e.value.status_name == "PF_ERR_STATE"
+    cache.rope_shift(0, pf.PART_SINK, 0)                         # a zero shift is a no-op
+    cache.append_block(0, blk["K"].cuda(), blk["V"].cuda())
+    cache.rope_shift(0, pf.PART_SINK, 4)
+    assert cache.info(0)["total_shift"] == 4
 
 
 # ------------------------------------------------------------------ failure detection
