@@ -454,7 +454,7 @@ def _timed(fn, iters, flush, stream):
 
 def run_suite(args):
     """One JSON line per hot-path kernel on the workload its roofline is
-    judged on: scoring and RoPE shift on the batch-2, 1,000-block stress
+    measured on: scoring and RoPE shift on the batch-2, 1,000-block stress
     layer (HBM-bound), attention on the layer / stress / dense workloads
     (tensor-bound), append, and the 30-layer block step."""
     import torch
