@@ -140,15 +140,27 @@ __device__ __forceinline__ SubBox decode_subbox(const AttendParams& p, int b, in
   return r;
 }
 
+// a mod b for 0 <= a < 2^22, 0 < b, with inv_b = 1 / b: a float estimate of
+// the quotient corrected by one step (cheaper than integer division on the
+// softmax's critical path).
+__device__ __forceinline__ int mod_small(int a, int b, float inv_b) {
+  int q = __float2int_rz(__int2float_rn(a) * inv_b);
+  int r = a - q * b;
+  if (r < 0) r += b;
+  else if (r >= b) r -= b;
+  return r;
+}
+
 // Valid rows of sub-box s (no table lookups: depends on the geometry only).
-__device__ __forceinline__ int subbox_valid(const AttendParams& p, int s) {
+// inv_mid / inv_blk = 1 / sb_mid, 1 / sb_blk.
+__device__ __forceinline__ int subbox_valid(const AttendParams& p, int s, float inv_mid, float inv_blk) {
   if (s < p.sb_sink) return min(kSub, p.sink_rows - s * kSub);
   s -= p.sb_sink;
   const int nmid = p.n_sel * p.sb_mid;
-  if (s < nmid) return min(kSub, p.n_c - (s % p.sb_mid) * kSub);
+  if (s < nmid) return min(kSub, p.n_c - mod_small(s, p.sb_mid, inv_mid) * kSub);
   s -= nmid;
   const int nrec = p.n_recent * p.sb_blk;
-  if (s < nrec) return min(kSub, p.n - (s % p.sb_blk) * kSub);
+  if (s < nrec) return min(kSub, p.n - mod_small(s, p.sb_blk, inv_blk) * kSub);
   s -= nrec;
   if (s < p.sb_blk) return min(kSub, p.n - s * kSub);
   return 0;
@@ -217,12 +229,13 @@ __device__ __forceinline__ float max64(const uint32_t* x) {
 // stored to 16 TMEM columns at dst; their sum accumulated in rs2.
 __device__ __forceinline__ void exp_chunk(const uint32_t* c, uint32_t dst, uint64_t sl2x2, uint64_t nmbx2,
                                           uint64_t* rs2) {
+  constexpr int period = kPolyPeriod > 0 ? kPolyPeriod : 1;
   uint32_t pk[16];
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
     const uint64_t x = f2_fma((static_cast<uint64_t>(c[2 * e + 1]) << 32) | c[2 * e], sl2x2, nmbx2);
     float p0, p1;
-    if (kPolyPeriod > 0 && (e % kPolyPeriod) == kPolyPeriod - 1) {
+    if (kPolyPeriod > 0 && (e % period) == period - 1) {
       p0 = ex2_poly(f2_lo(x));   // on the FMA pipe: unloads the special-function unit
       p1 = ex2_poly(f2_hi(x));
     } else {
@@ -528,6 +541,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
     const uint32_t tS = tmem + lane_off + t * 128u;
     const uint32_t tO = tmem + lane_off + 256u + t * 128u;
     const float sl2 = p.scale_log2;
+    const float inv_mid = 1.f / static_cast<float>(max(p.sb_mid, 1));
+    const float inv_blk = 1.f / static_cast<float>(max(p.sb_blk, 1));
     bool ok = t < nq;
     float m = -INFINITY;   // running max of scaled scores, base-2 units
     float l = 0.f;         // running sum of exp2(score - m)
@@ -541,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
       const bool check = !p.exact || (s0 + 4 > p.sb_mid_lo && s0 < p.sb_mid_hi) || (s0 + 4 > p.n_sub);
       if (check) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) valid[i] = subbox_valid(p, s0 + i);
+        for (int i = 0; i < 4; ++i) valid[i] = subbox_valid(p, s0 + i, inv_mid, inv_blk);
       }
       const bool masked = check && (valid[0] != kSub || valid[1] != kSub || valid[2] != kSub || valid[3] != kSub);
       // the whole row of S in registers: one tensor-memory round trip
@@ -549,7 +564,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
       tmem_ld128_wait(tS, sv);
       if (masked) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) mask32(sv + 32 * i, valid[i]);
+        for (int i = 0; i < 4; ++i)
+          if (valid[i] < kSub) mask32(sv + 32 * i, valid[i]);
       }
       const float mt = fmaxf(max64(sv), max64(sv + 64)) * sl2;
       float alpha = 1.f;
