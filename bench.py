@@ -274,29 +274,62 @@ def run_gpu(args):
     ms_per_step = total_ms / args.steps
     value = world * args.steps * flops / (total_ms * 1e-3) / 1e12
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers.  Each step's
+    # inputs come from pinned host memory and its output goes back to pinned
+    # host memory; the copies run on their own streams (host-to-device and
+    # device-to-host engines), double-buffered, so that step i+1's inputs and
+    # step i-1's output move while step i computes.  The timed region runs
+    # from before the first input copy to after the last output copy.
     pin = lambda t: t.cpu().pin_memory()  # noqa: E731
-    hQ, hK, hV, hKc, hVc = pin(Q), pin(Kn), pin(Vn), pin(Kcn), pin(Vcn)
-    hO = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
-    dQ, dK, dV, dKc, dVc = (torch.empty_like(t) for t in (Q, Kn, Vn, Kcn, Vcn))
-    h2d = sum(t.numel() * t.element_size() for t in (hQ, hK, hV, hKc, hVc))
-    d2h = hO.numel() * hO.element_size()
+    hin = tuple(pin(t) for t in (Q, Kn, Vn, Kcn, Vcn))
+    hO = [torch.empty(O.shape, dtype=O.dtype, pin_memory=True) for _ in range(2)]
+    din = [tuple(torch.empty_like(t) for t in (Q, Kn, Vn, Kcn, Vcn)) for _ in range(2)]
+    dO = [torch.empty_like(O) for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for t in hin)
+    d2h = hO[0].numel() * hO[0].element_size()
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    ev_in, ev_done, ev_out = [ev(), ev()], [ev(), ev()], [ev(), ev()]
 
-    def e2e_step():
-        for dst, src in ((dQ, hQ), (dK, hK), (dV, hV), (dKc, hKc), (dVc, hVc)):
-            dst.copy_(src, non_blocking=True)
-        step(dQ, dK, dV, dKc, dVc, O)
-        hO.copy_(O, non_blocking=True)
+    def e2e_run(nsteps, e_start=None, e_end=None):
+        if e_start is not None:
+            e_start.record(stream)
+        s_in.wait_stream(stream)
+        s_out.wait_stream(stream)
 
-    for _ in range(args.warmup):
-        e2e_step()
+        def copy_in(i):
+            b = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_done[b])        # step i-2 no longer reads these buffers
+                for dst, src in zip(din[b], hin):
+                    dst.copy_(src, non_blocking=True)
+                ev_in[b].record(s_in)
+
+        copy_in(0)
+        for i in range(nsteps):
+            b = i % 2
+            if i + 1 < nsteps:
+                copy_in(i + 1)
+            stream.wait_event(ev_in[b])
+            if i >= 2:
+                stream.wait_event(ev_out[b])           # step i-2's output has left dO[b]
+            step(*din[b], dO[b])
+            ev_done[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[b])
+                hO[b].copy_(dO[b], non_blocking=True)
+                ev_out[b].record(s_out)
+        stream.wait_stream(s_out)
+        stream.wait_stream(s_in)
+        if e_end is not None:
+            e_end.record(stream)
+
+    e2e_run(args.warmup)
     torch.cuda.synchronize(dev)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
+    e2e_run(args.steps, e0, e1)
     torch.cuda.synchronize(dev)
     barrier()
     e2e_ms = reduce_max(e0.elapsed_time(e1), dev)

@@ -72,8 +72,8 @@ constexpr bool kDrainBeforeOverwrite = PF_ATTEND_DRAIN != 0;
 #ifndef PF_ATTEND_MMA_POLL
 #define PF_ATTEND_MMA_POLL 0
 #endif
-// One exponential pair in kPolyPeriod is evaluated by ex2_poly (FMA pipe),
-// the others by the special-function unit (0 = never; measured slower).
+// One exponential pair in kPolyPeriod is evaluated by ex2_poly_x2 (FMA and
+// integer pipes), the others by the special-function unit (0 = never).
 #ifndef PF_ATTEND_POLY_PERIOD
 #define PF_ATTEND_POLY_PERIOD 0
 #endif
@@ -234,16 +234,13 @@ __device__ __forceinline__ void exp_chunk(const uint32_t* c, uint32_t dst, uint6
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
     const uint64_t x = f2_fma((static_cast<uint64_t>(c[2 * e + 1]) << 32) | c[2 * e], sl2x2, nmbx2);
-    float p0, p1;
-    if (kPolyPeriod > 0 && (e % period) == period - 1) {
-      p0 = ex2_poly(f2_lo(x));   // on the FMA pipe: unloads the special-function unit
-      p1 = ex2_poly(f2_hi(x));
-    } else {
-      p0 = ex2_approx(f2_lo(x));
-      p1 = ex2_approx(f2_hi(x));
-    }
-    rs2[e & 1] = f2_add(rs2[e & 1], f2_pack(p0, p1));
-    pk[e] = pack_bf16x2(p0, p1);
+    uint64_t pp;
+    if (kPolyPeriod > 0 && (e % period) == period - 1)
+      pp = ex2_poly_x2(x);   // FMA pipe: unloads the special-function unit
+    else
+      pp = f2_pack(ex2_approx(f2_lo(x)), ex2_approx(f2_hi(x)));
+    rs2[e & 1] = f2_add(rs2[e & 1], pp);
+    pk[e] = pack_bf16x2(f2_lo(pp), f2_hi(pp));
   }
   tmem_st16(dst, pk);
 }

@@ -270,6 +270,28 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// ex2_poly on both lanes of a pair: the rounding, the reduction and the
+// cubic as paired fp32 instructions, the exponent insertion as one
+// shift-and-add per lane.
+__device__ __forceinline__ uint64_t ex2_poly_x2(uint64_t x) {
+  x = f2_pack(fmaxf(f2_lo(x), -126.0f), fmaxf(f2_hi(x), -126.0f));
+  const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t t = f2_add(x, magic);
+  const uint64_t f = f2_sub(x, f2_sub(t, magic));
+  uint64_t p = f2_fma(f2_pack(5.517166906e-02f, 5.517166906e-02f), f, f2_pack(2.426111222e-01f, 2.426111222e-01f));
+  p = f2_fma(p, f, f2_pack(6.932609855e-01f, 6.932609855e-01f));
+  p = f2_fma(p, f, f2_pack(9.999280735e-01f, 9.999280735e-01f));
+  const uint32_t lo = static_cast<uint32_t>(p) + (static_cast<uint32_t>(t) << 23);
+  const uint32_t hi = static_cast<uint32_t>(p >> 32) + (static_cast<uint32_t>(t >> 32) << 23);
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
