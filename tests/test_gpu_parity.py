@@ -172,6 +172,51 @@ def test_selection_after_rotating_the_pool(pf, name):
             assert np.array_equal(sel.cpu().numpy()[b], sel_ref[b])
 
 
+def test_largest_pool_selection_and_attention(pf):
+    # the largest pool a cache allows (8,192 slots = 8,191 live blocks + the
+    # recent block's pending copy): the top-k keeps every score in shared memory
+    wl = _wl("tiny").replace(mid_capacity=8191, pool_blocks=8191, planted=16, n_top=16)
+    d = synth.make_layer(wl, 31)
+    cache = build_cache(pf, wl, d)
+    assert cache.info(0)["pool_slots"] == 8192 and cache.info(0)["mid_count"] == 8191
+    Q = d["Q"].cuda()
+    sel = torch.full((1, 16), -1, dtype=torch.int32, device="cuda")
+    sc = torch.zeros((1, 8191), dtype=torch.float32, device="cuda")
+    cache.select_mid(0, Q, sel, sc)
+    O = cache.attend(0, Q, d["K_cur"].cuda(), d["V_cur"].cuda())
+    torch.cuda.synchronize()
+    S_ref = oracle.select_scores(d["Q"], d["mid_K"])
+    assert oracle.selection_margin(S_ref, 16)[0] >= 1e-3
+    assert np.array_equal(sel.cpu().numpy(), oracle.select_topk(S_ref, 16))
+    assert np.max(np.abs(sc.cpu().numpy() - S_ref)) < 1e-4 * np.abs(S_ref).max()
+    O_ref, _ = oracle.attend(d["Q"], oracle_context(wl, d, sel.cpu().numpy()))
+    assert_attention_close(O.cpu(), O_ref, "8,191-block pool")
+
+
+def test_large_top_k_is_a_valid_selection(pf):
+    # n_top = 3,000 of 8,191 random scores: no margin, so check what is unique
+    # (the selected set is the 3,000 largest GPU scores, ties to the older
+    # block) and that the scores match the oracle
+    wl = _wl("tiny").replace(mid_capacity=8191, pool_blocks=8191, planted=0, n_top=3000)
+    d = synth.make_layer(wl, 32)
+    cache = build_cache(pf, wl, d)
+    sel = torch.full((1, 3000), -1, dtype=torch.int32, device="cuda")
+    sc = torch.zeros((1, 8191), dtype=torch.float32, device="cuda")
+    cache.select_mid(0, d["Q"].cuda(), sel, sc)
+    torch.cuda.synchronize()
+    s = sel.cpu().numpy()[0]
+    g = sc.cpu().numpy()[0]
+    assert np.all(np.diff(s) > 0) and s[0] >= 0 and s[-1] < 8191          # ascending, distinct
+    chosen = np.zeros(8191, dtype=bool)
+    chosen[s] = True
+    T = g[chosen].min()
+    assert g[~chosen].max() <= T                                             # the largest scores
+    eq = np.flatnonzero(g == T)
+    assert np.all(chosen[eq[:chosen[eq].sum()]]) and not np.any(chosen[eq[chosen[eq].sum():]])   # older first
+    S_ref = oracle.select_scores(d["Q"], d["mid_K"])[0]
+    assert np.max(np.abs(g - S_ref)) < 1e-4 * np.abs(S_ref).max()
+
+
 def test_selection_ties_go_to_older_blocks(pf):
     wl = _wl("ragged_a").replace(pool_blocks=9, planted=0, mid_capacity=9, n_top=4)
     d = synth.make_layer(wl, 5)
