@@ -72,6 +72,17 @@ constexpr bool kDrainBeforeOverwrite = PF_ATTEND_DRAIN != 0;
 #ifndef PF_ATTEND_MMA_POLL
 #define PF_ATTEND_MMA_POLL 0
 #endif
+// The two query tiles' exponential phases alternate: tile 1's for K/V tile j
+// starts once tile 0's P_j is ready, tile 0's for tile j+1 once tile 1's P_j
+// is.  Their softmaxes then share the special-function unit in turns and
+// each tile's MMAs run during the other tile's softmax.  Without the gate
+// the two tiles can fall into step (after a run of masked tiles, or from the
+// start): both softmaxes contend for the unit and both tiles' MMAs queue
+// back to back (~1.5x the time per K/V tile).
+#ifndef PF_ATTEND_SLOT_GATE
+#define PF_ATTEND_SLOT_GATE 0
+#endif
+constexpr bool kSlotGate = PF_ATTEND_SLOT_GATE != 0;
 // One exponential pair in kPolyPeriod is evaluated by ex2_poly_x2 (FMA and
 // integer pipes), the others by the special-function unit (0 = never).
 #ifndef PF_ATTEND_POLY_PERIOD
@@ -100,13 +111,27 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
 
+// floor(a / b) and a mod b for 0 <= a < 2^22, 0 < b, with inv_b = 1 / b: a
+// float estimate of the quotient corrected by one step (integer division by
+// a run-time value is a long instruction sequence, costly on the producer's
+// and the softmax's paths).
+__device__ __forceinline__ int div_small(int a, int b, float inv_b) {
+  int q = __float2int_rz(__int2float_rn(a) * inv_b);
+  const int r = a - q * b;
+  if (r < 0) --q;
+  else if (r >= b) ++q;
+  return q;
+}
+__device__ __forceinline__ int mod_small(int a, int b, float inv_b) { return a - div_small(a, b, inv_b) * b; }
+
 struct SubBox {
   int part, row0, seg, valid;
 };
 
 // Sub-box s of batch item b's context: which partition, first row, segment
 // (index along the tensor map's outermost dimension), and valid rows.
-__device__ __forceinline__ SubBox decode_subbox(const AttendParams& p, int b, int s) {
+// inv_mid / inv_blk = 1 / sb_mid, 1 / sb_blk.
+__device__ __forceinline__ SubBox decode_subbox(const AttendParams& p, int b, int s, float inv_mid, float inv_blk) {
   SubBox r;
   if (s < p.sb_sink) {
     r.part = kPartSink; r.row0 = s * kSub; r.seg = b; r.valid = min(kSub, p.sink_rows - r.row0);
@@ -115,8 +140,14 @@ __device__ __forceinline__ SubBox decode_subbox(const AttendParams& p, int b, in
   s -= p.sb_sink;
   const int nmid = p.n_sel * p.sb_mid;
   if (s < nmid) {
-    const int blk = s / p.sb_mid, k = s - blk * p.sb_mid;
-    const int slot = p.sel_slots ? p.sel_slots[b * p.sel_stride + blk] : (p.mid_head + blk) % p.pool_slots;
+    const int blk = div_small(s, p.sb_mid, inv_mid), k = s - blk * p.sb_mid;
+    int slot;
+    if (p.sel_slots) {
+      slot = p.sel_slots[b * p.sel_stride + blk];
+    } else {
+      slot = p.mid_head + blk;   // < 2 pool_slots
+      if (slot >= p.pool_slots) slot -= p.pool_slots;
+    }
     r.part = kPartMid; r.row0 = k * kSub; r.seg = b * p.pool_slots + slot;
     r.valid = min(kSub, p.n_c - r.row0);
     return r;
@@ -124,8 +155,9 @@ __device__ __forceinline__ SubBox decode_subbox(const AttendParams& p, int b, in
   s -= nmid;
   const int nrec = p.n_recent * p.sb_blk;
   if (s < nrec) {
-    const int blk = s / p.sb_blk, k = s - blk * p.sb_blk;
-    const int slot = (p.recent_head + blk) % p.recent_slots;
+    const int blk = div_small(s, p.sb_blk, inv_blk), k = s - blk * p.sb_blk;
+    int slot = p.recent_head + blk;   // < 2 recent_slots
+    if (slot >= p.recent_slots) slot -= p.recent_slots;
     r.part = kPartRecent; r.row0 = k * kSub; r.seg = b * p.recent_slots + slot;
     r.valid = min(kSub, p.n - r.row0);
     return r;
@@ -137,17 +169,6 @@ __device__ __forceinline__ SubBox decode_subbox(const AttendParams& p, int b, in
   }
   // padding past the end of the context: a box fully outside the map, zero-filled
   r.part = kPartCur; r.row0 = ((p.n + kSub - 1) / kSub) * kSub; r.seg = b; r.valid = 0;
-  return r;
-}
-
-// a mod b for 0 <= a < 2^22, 0 < b, with inv_b = 1 / b: a float estimate of
-// the quotient corrected by one step (cheaper than integer division on the
-// softmax's critical path).
-__device__ __forceinline__ int mod_small(int a, int b, float inv_b) {
-  int q = __float2int_rz(__int2float_rn(a) * inv_b);
-  int r = a - q * b;
-  if (r < 0) r += b;
-  else if (r >= b) r -= b;
   return r;
 }
 
@@ -320,6 +341,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
           tma_load_4d(smem + kOffQ + t * kTileBytes + half * kHalfBytes, &p.tm_q, &bars.q_full, half * 64,
                       un.t[t].h, un.t[t].qt * kBM, un.t[t].b);
       const int b = un.t[0].b, h = un.t[0].h;
+      const float inv_mid = 1.f / static_cast<float>(max(p.sb_mid, 1));
+      const float inv_blk = 1.f / static_cast<float>(max(p.sb_blk, 1));
       int kg = 0, vg = 0;    // K / V tiles issued
       bool ok = true;
       for (int j = un.j0; ok && j < un.j1; ++j) {
@@ -332,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
           }
           mbar_arrive_expect_tx(&bars.k_full[st], kTileBytes);
           for (int i = 0; i < 4; ++i) {
-            const SubBox sb = decode_subbox(p, b, 4 * j + i);
+            const SubBox sb = decode_subbox(p, b, 4 * j + i, inv_mid, inv_blk);
             for (int half = 0; half < 2; ++half)
               tma_load_4d(smem + kOffK + st * kTileBytes + half * kHalfBytes + i * kSubBytes, &p.tm_k[sb.part],
                           &bars.k_full[st], half * 64, h, sb.row0, sb.seg);
@@ -348,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
           }
           mbar_arrive_expect_tx(&bars.v_full[st], kTileBytes);
           for (int i = 0; i < 4; ++i) {
-            const SubBox sb = decode_subbox(p, b, 4 * j + i);
+            const SubBox sb = decode_subbox(p, b, 4 * j + i, inv_mid, inv_blk);
             for (int half = 0; half < 2; ++half)
               tma_load_4d(smem + kOffV + st * kTileBytes + half * kHalfBytes + i * kSubBytes, &p.tm_v[sb.part],
                           &bars.v_full[st], half * 64, h, sb.row0, sb.seg);
@@ -572,6 +595,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
         l *= alpha;
         rescale_o = j > un.j0;
         m = mt;
+      }
+      if (kSlotGate && nq == 2 && (t == 1 || j > un.j0)) {
+        // take turns with the other query tile (see kSlotGate)
+        const int o = t ^ 1, jj = (t == 1) ? j : j - 1;
+        ok = mbar_wait_bounded(&bars.p_full[o], (jj - un.j0) & 1, abort_flag, p.err, kDevErrTimeoutBase | 15u, lim);
+        if (!ok) break;
       }
       const float mb = (m == -INFINITY) ? 0.f : m;
       const uint64_t sl2x2 = f2_pack(sl2, sl2), nmbx2 = f2_pack(-mb, -mb);
