@@ -567,10 +567,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
     float m = -INFINITY;   // running max of scaled scores, base-2 units
     float l = 0.f;         // running sum of exp2(score - m)
     for (int j = un.j0; ok && j < un.j1; ++j) {
-      ok = mbar_wait_bounded(&bars.s_full[t], (j - un.j0) & 1, abort_flag, p.err, kDevErrTimeoutBase | 11u, lim);
-      if (!ok) break;
-      tc_fence_after();
-      // which columns hold real keys (most tiles: all of them)
+      // which columns hold real keys (most tiles: all of them); worked out
+      // before S is ready, off the critical path
       const int s0 = 4 * j;
       int valid[4] = {kSub, kSub, kSub, kSub};
       const bool check = !p.exact || (s0 + 4 > p.sb_mid_lo && s0 < p.sb_mid_hi) || (s0 + 4 > p.n_sub);
@@ -579,6 +577,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
         for (int i = 0; i < 4; ++i) valid[i] = subbox_valid(p, s0 + i, inv_mid, inv_blk);
       }
       const bool masked = check && (valid[0] != kSub || valid[1] != kSub || valid[2] != kSub || valid[3] != kSub);
+      ok = mbar_wait_bounded(&bars.s_full[t], (j - un.j0) & 1, abort_flag, p.err, kDevErrTimeoutBase | 11u, lim);
+      if (!ok) break;
+      tc_fence_after();
       // the whole row of S in registers: one tensor-memory round trip
       uint32_t sv[128];
       tmem_ld128_wait(tS, sv);
