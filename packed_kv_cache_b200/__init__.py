@@ -72,7 +72,20 @@ class LayerInfo(ctypes.Structure):
         return {name: getattr(self, name) for name, _ in self._fields_}
 
 
+def _build_from_sources() -> None:
+    """A checkout without the built library but with its sources: compile it
+    (nvcc, sm_100a) before loading.  build.py is loaded by path so that this
+    package is not imported again; a failed build raises."""
+    from importlib.util import module_from_spec, spec_from_file_location
+    spec = spec_from_file_location("_packed_kv_cache_b200_build", os.path.join(_HERE, "build.py"))
+    mod = module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+
+
 def _load():
+    if not os.path.exists(library_path) and os.path.isdir(os.path.join(_HERE, "csrc")):
+        _build_from_sources()
     if not os.path.exists(library_path):
         raise ImportError(f"{library_path} is missing: build it with `python -m packed_kv_cache_b200.build`")
     L = ctypes.CDLL(library_path)
