@@ -113,6 +113,34 @@ def test_calls_reject_null_cache(pf):
     assert pf.lib.pf_poll_device_error(None, None, None) == 1
 
 
+def test_static_selection_checks_arguments_before_device_work(pf):
+    # placeholder device addresses: every case below returns before the library
+    # touches them (argument and capacity checks, or nothing to select)
+    Q, K, sel = 0x100000, 0x200000, 0x300000
+    f = pf.lib.pf_select_mid_static
+    LIMITS = {k: int(v) for k, v in re.findall(r"#define (PF_STATIC_MAX_\w+) (\d+)", open(HEADER).read())}
+    assert len(LIMITS) == 4
+
+    def call(Q=Q, batch=1, n=64, heads=1, K=K, slots=8, n_c=4, head=0, count=8, n_top=4, sel=sel, scores=None):
+        return f(Q, batch, n, heads, K, slots, n_c, head, count, n_top, sel, scores, None)
+
+    assert call(Q=None) == 1 and call(K=None) == 1 and call(sel=None) == 1
+    assert call(Q=Q + 8) == 1 and b"misaligned" in pf.lib.pf_last_error()
+    assert call(sel=sel + 2) == 1 and call(scores=0x400002) == 1
+    assert call(n=0) == 1 and call(n_c=0) == 1 and call(count=-1) == 1 and call(n_top=-1) == 1
+    assert call(slots=4, count=8) == 1      # more live blocks than slots
+    assert call(head=8) == 1 and call(head=-1) == 1
+    # capacity of the fixed scratch array
+    assert call(batch=LIMITS["PF_STATIC_MAX_BATCH"] + 1) == 4
+    assert call(heads=LIMITS["PF_STATIC_MAX_HEADS"] + 1) == 4
+    assert call(slots=LIMITS["PF_STATIC_MAX_BLOCKS"] + 1,
+                count=LIMITS["PF_STATIC_MAX_BLOCKS"] + 1) == 4
+    assert call(n_c=LIMITS["PF_STATIC_MAX_NC"] + 1) == 4
+    assert call(batch=8, slots=4097) == 4 and b"pool_slots" in pf.lib.pf_last_error()
+    # nothing to select: success with no device work
+    assert call(count=0) == 0 and call(n_top=0) == 0
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     # importing the binding from a copy without libpf.so must raise, not fall back
     import shutil
