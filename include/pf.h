@@ -114,7 +114,9 @@ const char* pf_status_string(pf_status s);
  * follow PackForcing (arXiv), "KV Caching" (n = B_f h w) and "Compressed Mid
  * Tokens" (n_c = floor(B_f/2) floor(h/4) floor(w/4)).
  * Errors: PF_ERR_ARG for a null pointer or a non-positive size,
- * PF_ERR_UNSUPPORTED for head_dim != 128 or rope_split not summing to it.
+ * PF_ERR_UNSUPPORTED for head_dim != 128 or rope_split not summing to it,
+ * PF_ERR_CAPACITY when a size limit is exceeded or the total does not fit
+ * in size_t.
  */
 pf_status pf_cache_bytes(const pf_config* cfg, size_t* bytes);
 
@@ -123,7 +125,8 @@ pf_status pf_cache_bytes(const pf_config* cfg, size_t* bytes);
  * 256-byte aligned.  Zeroes the arena on `stream` (asynchronously).  The
  * arena must outlive the cache; pf_cache_destroy frees only host state.
  * Errors: PF_ERR_ARG, PF_ERR_ARENA (too small / misaligned), PF_ERR_UNSUPPORTED,
- * PF_ERR_CUDA.
+ * PF_ERR_CAPACITY (as pf_cache_bytes; or no host memory for the layers'
+ * state), PF_ERR_CUDA.
  */
 pf_status pf_cache_create(const pf_config* cfg, void* dev_arena, size_t arena_bytes,
                           void* stream, pf_cache** out);

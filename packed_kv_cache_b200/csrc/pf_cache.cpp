@@ -55,7 +55,7 @@ struct Geometry {
   int n, n_c, slots, HD;
   size_t sink_bytes, pool_bytes, recent_bytes;  // per K (or V) tensor
   size_t sel_bytes, scores_bytes, partial_bytes, qsum_bytes, ticket_bytes, kbar_bytes;
-  size_t layer_bytes;
+  size_t layer_bytes, arena_bytes;
   int chunk_rows, chunks_per_block;
 };
 
@@ -85,8 +85,29 @@ pf_status check_config(const pf_config* c) {
   return PF_OK;
 }
 
-Geometry geometry(const pf_config* c) {
+// Size arithmetic that records an overflow instead of wrapping around: a
+// wrapped arena size would let the partitions of a huge configuration be
+// laid out past the end of the caller's arena.
+struct Sizes {
+  bool overflow = false;
+  size_t mul(size_t a, size_t b) {
+    size_t r = 0;
+    if (__builtin_mul_overflow(a, b, &r)) overflow = true;
+    return r;
+  }
+  size_t add(size_t a, size_t b) {
+    size_t r = 0;
+    if (__builtin_add_overflow(a, b, &r)) overflow = true;
+    return r;
+  }
+  size_t aligned(size_t x) { return mul(add(x, kAlign - 1) / kAlign, kAlign); }
+  size_t bytes(size_t a, size_t b, size_t c, size_t d = 1) { return aligned(mul(mul(a, b), mul(c, d))); }
+};
+
+// Sets *overflow when a size does not fit in size_t.
+Geometry geometry(const pf_config* c, bool* overflow) {
   Geometry g;
+  Sizes z;
   g.n = c->block_frames * c->h * c->w;
   g.n_c = (c->block_frames / 2) * (c->h / 4) * (c->w / 4);
   if (g.n_c < 1) g.n_c = 1;  // pool unused (mid_capacity == 0); keep the maps well formed
@@ -94,19 +115,23 @@ Geometry geometry(const pf_config* c) {
   g.HD = c->heads * c->head_dim;
   const size_t row = static_cast<size_t>(g.HD) * 2;
   const size_t B = static_cast<size_t>(c->batch);
-  g.sink_bytes = align_up(B * c->sink_blocks * g.n * row);
-  g.pool_bytes = align_up(B * g.slots * g.n_c * row);
-  g.recent_bytes = align_up(B * c->recent_blocks * g.n * row);
+  g.sink_bytes = z.bytes(B, c->sink_blocks, g.n, row);
+  g.pool_bytes = z.bytes(B, g.slots, g.n_c, row);
+  g.recent_bytes = z.bytes(B, c->recent_blocks, g.n, row);
   g.chunk_rows = 32;
   g.chunks_per_block = (g.n_c + g.chunk_rows - 1) / g.chunk_rows;
-  g.sel_bytes = align_up(B * (c->n_top > 0 ? c->n_top : 1) * 4);
-  g.scores_bytes = align_up(B * g.slots * 4);
-  g.partial_bytes = align_up(B * g.slots * g.chunks_per_block * 4);
-  g.qsum_bytes = align_up(B * g.HD * 4);
-  g.ticket_bytes = align_up(B * 4);
-  g.kbar_bytes = align_up(B * g.slots * g.HD * 4);
-  g.layer_bytes = 2 * (g.sink_bytes + g.pool_bytes + g.recent_bytes) + g.sel_bytes + g.scores_bytes +
-                  g.partial_bytes + g.qsum_bytes + g.ticket_bytes + g.kbar_bytes;
+  g.sel_bytes = z.bytes(B, c->n_top > 0 ? c->n_top : 1, 4);
+  g.scores_bytes = z.bytes(B, g.slots, 4);
+  g.partial_bytes = z.bytes(B, g.slots, g.chunks_per_block, 4);
+  g.qsum_bytes = z.bytes(B, g.HD, 4);
+  g.ticket_bytes = z.bytes(B, 4, 1);
+  g.kbar_bytes = z.bytes(B, g.slots, g.HD, 4);
+  size_t t = z.mul(2, z.add(z.add(g.sink_bytes, g.pool_bytes), g.recent_bytes));
+  t = z.add(t, z.add(z.add(g.sel_bytes, g.scores_bytes), g.partial_bytes));
+  t = z.add(t, z.add(z.add(g.qsum_bytes, g.ticket_bytes), g.kbar_bytes));
+  g.layer_bytes = t;
+  g.arena_bytes = z.add(kAlign /* error word */ + kAttendScratchBytes, z.mul(g.layer_bytes, c->layers));
+  *overflow = z.overflow;
   return g;
 }
 
@@ -277,8 +302,10 @@ pf_status pf_cache_bytes(const pf_config* cfg, size_t* bytes) {
   pf_status s = check_config(cfg);
   if (s != PF_OK) return s;
   if (bytes == nullptr) return fail(PF_ERR_ARG, "bytes is NULL");
-  const Geometry g = geometry(cfg);
-  *bytes = kAlign /* error word */ + kAttendScratchBytes + g.layer_bytes * static_cast<size_t>(cfg->layers);
+  bool overflow = false;
+  const Geometry g = geometry(cfg, &overflow);
+  if (overflow) return fail(PF_ERR_CAPACITY, "the cache's size does not fit in size_t");
+  *bytes = g.arena_bytes;
   return PF_OK;
 }
 
@@ -293,12 +320,18 @@ pf_status pf_cache_create(const pf_config* cfg, void* dev_arena, size_t arena_by
   pf_cache* c = new (std::nothrow) pf_cache();
   if (c == nullptr) return fail(PF_ERR_CAPACITY, "out of host memory");
   c->cfg = *cfg;
-  c->g = geometry(cfg);
+  bool overflow = false;
+  c->g = geometry(cfg, &overflow);  // no overflow: pf_cache_bytes succeeded
   c->arena = static_cast<char*>(dev_arena);
   c->arena_bytes = arena_bytes;
   c->err = reinterpret_cast<unsigned*>(c->arena);
   c->timeout_cycles = kDefaultTimeoutCycles;
-  c->L.resize(cfg->layers);
+  try {
+    c->L.resize(cfg->layers);
+  } catch (...) {  // no exception may cross the C ABI
+    delete c;
+    return fail(PF_ERR_CAPACITY, "out of host memory for %d layers", cfg->layers);
+  }
   char* p = c->arena + kAlign;
   c->part_o = reinterpret_cast<float*>(p); p += pf::kAttendPartOBytes;
   c->part_ml = reinterpret_cast<float*>(p); p += pf::kAttendPartMLBytes;

@@ -86,6 +86,22 @@ def test_config_validation(pf, field, value, status):
     assert e.value.status_name == status
 
 
+def test_cache_bytes_reports_overflow_instead_of_wrapping(pf):
+    # 2^31 batch items x 2^31 sink blocks x 2^24 tokens x 128 KB rows is far
+    # past size_t: the size must be refused, never wrapped to a small arena
+    big = dict(batch=2**31 - 1, sink_blocks=2**31 - 1, heads=512, block_frames=2, h=4096, w=2048)
+    with pytest.raises(pf.PFError) as e:
+        pf.pf_cache_bytes(_cfg(pf, **big))
+    assert e.value.status_name == "PF_ERR_CAPACITY"
+    assert b"size_t" in pf.lib.pf_last_error()
+    # create refuses it the same way, before looking at the arena
+    h = ctypes.c_void_p()
+    assert pf.lib.pf_cache_create(ctypes.byref(_cfg(pf, **big)), 0x100000, 2**63, None, ctypes.byref(h)) == 4
+    # the largest sizes that still fit are computed exactly
+    one, two = (pf.pf_cache_bytes(_cfg(pf, layers=k)) for k in (1, 2))
+    assert pf.pf_cache_bytes(_cfg(pf, layers=2**31 - 1)) == one + (2**31 - 2) * (two - one)
+
+
 def test_rope_split_validation(pf):
     c = _cfg(pf)
     c.rope_split[0] = 46
