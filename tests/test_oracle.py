@@ -177,6 +177,20 @@ def test_planted_blocks_recovered_tiny():
     assert oracle.selection_margin(S, 3)[0] >= 1e-3
 
 
+@pytest.mark.parametrize("name", ["tiny", "ragged_a", "ragged_b", "ragged_c", "layer", "step30"])
+def test_stored_seeds_plant_the_oracle_top_k(name):
+    # the seed fixture still holds for the generator and the oracle as they are:
+    # planted blocks = the oracle's top-k in every batch item, at the stored margin
+    seeds = _gold("seeds.json")
+    wl = synth.WORKLOADS[name]
+    d = synth.make_layer(wl, seeds[name], with_values=False)
+    S = oracle.select_scores(d["Q"], d["mid_K"])
+    assert np.array_equal(oracle.select_topk(S, wl.n_top), d["planted"].numpy())
+    margin = oracle.selection_margin(S, wl.n_top)
+    assert np.all(margin >= 1e-3)
+    assert round(float(margin.min()), 4) == seeds["_margins"][name]
+
+
 def test_selection_permutation_equivariance():
     d = _tiny()
     S = oracle.select_scores(d["Q"], d["mid_K"])
