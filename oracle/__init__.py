@@ -98,12 +98,18 @@ def compressed_tokens_latent(T: int, H: int, W: int) -> int:
 
 
 def dense_context_tokens(blocks: int, n: int) -> int:
-    """Full, uncompressed context of ``blocks`` generated blocks."""
+    """Full, uncompressed context of ``blocks`` generated blocks: the growth
+    the pages quote as about 749K tokens for a 2-minute 832x480 16-FPS video
+    (PackForcing digest, KV-cache paragraph; the blog post "PackForcing:
+    Rethinking the Training-Generation Length Paradigm in Video Diffusion",
+    "The Memory Wall in Autoregressive Video Generation")."""
     return blocks * n
 
 
 def kv_bytes(tokens: int, hidden: int, layers: int, bytes_per_elem: int = 2) -> int:
-    """Bytes of K and V for ``tokens`` tokens over ``layers`` layers."""
+    """Bytes of K and V for ``tokens`` tokens over ``layers`` layers: the
+    pages' roughly 138 GB for that full context over 30 layers (same passages
+    as ``dense_context_tokens``)."""
     return tokens * hidden * 2 * bytes_per_elem * layers
 
 
@@ -232,7 +238,10 @@ def select_fifo(count: int, n_top: int) -> np.ndarray:
 def select_scores_bruteforce(Q, pool_K) -> np.ndarray:
     """The same scores as the token-level double sum sum_i sum_j q_i . k_j.
 
-    Small inputs only: one explicit q_i . k_j dot product per (i, j, h).
+    The digest's affinity phi_j = sum_i q_i^T k_j / sqrt(d) (PackForcing
+    digest, step (3)) written out term by term, summed over the block's keys
+    and averaged over heads and queries as in ``select_scores``.  Small inputs
+    only: one explicit q_i . k_j dot product per (i, j, h).
     """
     q = to_f64(Q)
     k = to_f64(pool_K)
@@ -270,7 +279,9 @@ def select_topk(scores, n_top: int) -> np.ndarray:
 def selection_margin(scores, n_top: int) -> np.ndarray:
     """Relative gap (S_(k) - S_(k+1)) / max_p |S_p| per row, k = n_top.
 
-    Infinite when every block is selected.
+    Not a step of the method: the gap that decides when a selection is far
+    enough from a tie for an exact comparison (the selection margin's reading
+    as a scale-free gap).  Infinite when every block is selected.
     """
     S = np.asarray(scores, dtype=np.float64)
     B, P = S.shape
@@ -332,7 +343,9 @@ def attend(Q, parts, scale=None, rows=None, chunk: int = 256):
 def attend_loops(Q, K, V, scale=None):
     """Brute-force twin of ``attend`` on one explicit K/V: plain loops.
 
-    Tiny inputs only.  Q [Lq, D], K [Lk, D], V [Lk, D] for one head.
+    The attention of the digest's KV-cache paragraph, softmax(Q K^T /
+    sqrt(d_h)) V, one explicit sum per query, key and dim.  Tiny inputs only.
+    Q [Lq, D], K [Lk, D], V [Lk, D] for one head.
     """
     q, k, v = to_f64(Q), to_f64(K), to_f64(V)
     Lq, D = q.shape
@@ -354,6 +367,9 @@ def attend_loops(Q, K, V, scale=None):
 def merge_partials(outs, lses):
     """Combine attention results over disjoint key sets by their LSEs.
 
+    Not a step the pages state: the identity that softmax attention over a
+    union of disjoint key sets is the LSE-weighted mix of the attention over
+    each set, used to check the partitioned form against the concatenated one.
     O = sum_j exp(lse_j - lse) O_j with lse = log sum_j exp(lse_j).
     outs: list of [B, Lq, H, D]; lses: list of [B, H, Lq].
     """
