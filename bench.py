@@ -389,18 +389,25 @@ def run_gpu(args):
 
 # ---------------------------------------------------------------- the oracle on host cores
 
-def oracle_step(d, wl, rows):
+def oracle_step(d, wl, rows, heads=None):
     """One bounded sample of the step on the CPU oracle: selection over the
-    whole pool, the sink shift, and attention for ``rows`` query rows."""
+    whole pool, the sink shift, and attention for ``rows`` query rows; with
+    ``heads`` = (lo, hi), every part restricted to those heads (the inputs are
+    sliced before the oracle sees them)."""
+    import numpy as np
+
     import oracle
+    if heads is not None:
+        lo, hi = heads
+        d = {k: (v[..., lo:hi, :] if hasattr(v, "dim") and v.dim() >= 4 else v) for k, v in d.items()}
     S = oracle.select_scores(d["Q"], d["mid_K"])
     sel = oracle.select_topk(S, wl.n_top)
-    B, H, D = wl.batch, wl.heads, wl.head_dim
+    B, D = wl.batch, wl.head_dim
+    H = d["Q"].shape[2]
     sinkK = oracle.rope_shift(d["sink_K"].reshape(B, -1, H, D), wl.block_frames)
     parts = [(sinkK, d["sink_V"].reshape(B, -1, H, D))]
     mK = [oracle.to_f64(d["mid_K"][b, sel[b]]).reshape(-1, H, D) for b in range(B)]
     mV = [oracle.to_f64(d["mid_V"][b, sel[b]]).reshape(-1, H, D) for b in range(B)]
-    import numpy as np
     parts.append((np.stack(mK), np.stack(mV)))
     parts.append((d["recent_K"].reshape(B, -1, H, D), d["recent_V"].reshape(B, -1, H, D)))
     parts.append((d["K_cur"], d["V_cur"]))
@@ -442,13 +449,43 @@ def run_reference(args):
         return
     wl = synth.WORKLOADS[WORKLOAD]
     d = synth.make_layer(wl, synth.nominal_seed(list(synth.WORKLOADS).index(WORKLOAD)))
-    rows = np.linspace(0, wl.n - 1, args.ref_rows).astype(np.int64)
+
+    def sample_rows(nr):
+        return np.linspace(0, wl.n - 1, nr).astype(np.int64)
+
+    if args.ref_rows:
+        nh, nr = wl.heads, args.ref_rows
+    else:
+        # size the per-step sample so that the warm-up and timed steps fit in
+        # --ref-seconds whatever --steps is: start from one head and 16 query
+        # rows, then double the heads (up to all of them), else the rows, as
+        # long as one measured step of the larger sample still fits
+        def step_seconds(nh, nr):
+            t0 = time.perf_counter()
+            oracle_step(d, wl, sample_rows(nr), (0, nh))
+            return time.perf_counter() - t0
+
+        per_step = args.ref_seconds / (args.steps + args.warmup)
+        nh, nr = 1, 16
+        t = step_seconds(nh, nr)
+        while t < per_step:
+            for cand in ((min(wl.heads, 2 * nh), nr), (nh, min(wl.n, 2 * nr))):
+                if cand == (nh, nr):
+                    continue
+                tc = step_seconds(*cand)
+                if tc <= per_step:
+                    (nh, nr), t = cand, tc
+                    break
+            else:
+                break
+    rows = sample_rows(nr)
+    heads = (0, nh)
     for _ in range(args.warmup):
-        oracle_step(d, wl, rows)
+        oracle_step(d, wl, rows, heads)
     t0 = time.perf_counter()
     fl = 0.0
     for _ in range(args.steps):
-        fl += oracle_step(d, wl, rows)
+        fl += oracle_step(d, wl, rows, heads)
     dt = time.perf_counter() - t0
     v = fl / dt / 1e12
     line = {
@@ -459,10 +496,11 @@ def run_reference(args):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": ("one layer, pages scale: B=1, H=12, d_h=128, n=6240, pool 40x182, "
                                 "top-16, context 27872 keys; oracle sample per step"),
-                   "rows_per_step": int(args.ref_rows)},
+                   "rows_per_step": int(nr), "heads_per_step": int(nh)},
         "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
-                         "sample": f"per step: selection over the whole pool, sink shift, attention of "
-                                   f"{args.ref_rows} of 6240 query rows x 12 heads"},
+                         "sample": f"per step, on {nh} of {wl.heads} heads: selection over the whole pool, "
+                                   f"sink shift, attention of {nr} of {wl.n} query rows over the "
+                                   f"27872-key context; float64 numpy"},
         "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -648,7 +686,10 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
-    ap.add_argument("--ref-rows", type=int, default=24)
+    ap.add_argument("--ref-rows", type=int, default=0,
+                    help="reference arm: query rows per step on all heads (default: sized to --ref-seconds)")
+    ap.add_argument("--ref-seconds", type=float, default=120.0,
+                    help="reference arm: host seconds for the warm-up and timed steps together")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--suite", action="store_true",
