@@ -422,12 +422,12 @@ def cpu_baseline(d, wl, budget_s=15.0):
     # two short calibrations separate the fixed cost (selection over the
     # pool, sink shift) from the per-query-row cost of the attention sample
     times = []
-    for nr in (16, 64):
+    for nr in (16, 256):
         rows = np.linspace(0, wl.n - 1, nr).astype(np.int64)
         t0 = time.perf_counter()
         oracle_step(dc, wl, rows)
         times.append(time.perf_counter() - t0)
-    per_row = max((times[1] - times[0]) / 48, 1e-6)
+    per_row = max((times[1] - times[0]) / 240, 1e-6)
     fixed = max(times[0] - 16 * per_row, 0.0)
     nrows = int(min(wl.n, max(16, (0.9 * budget_s - fixed) / per_row)))
     rows = np.linspace(0, wl.n - 1, nrows).astype(np.int64)
