@@ -128,34 +128,43 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        import datetime
-        rows = []
         with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
-                except ValueError:
-                    ts = None
-                if t0 is not None and ts is not None and not (t0 <= ts <= t1):
-                    continue
-                rows.append(parts)
+            lines = f.readlines()
         os.unlink(self.path)
-        if not rows:
+        return summarize_clocks(lines, t0, t1)
+
+
+def summarize_clocks(lines, t0: float | None = None, t1: float | None = None):
+    """Median SM clock, max clock and active throttle reasons of nvidia-smi
+    CSV rows (the ClockSampler fields, no header, no units) whose timestamp
+    lies in [t0, t1] (host time); None if no row qualifies."""
+    import datetime
+    rows = []
+    for line in lines:
+        parts = [x.strip() for x in line.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            ts = None
+        if t0 is not None and ts is not None and not (t0 <= ts <= t1):
+            continue
+        rows.append(parts)
+    if not rows:
+        return None
+
+    def num(x):
+        try:
+            return float(x)
+        except ValueError:
             return None
-        def num(x):
-            try:
-                return float(x)
-            except ValueError:
-                return None
-        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
-        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+    sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+    mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+            "reasons": reasons, "samples": len(rows)}
 
 
 def traffic_for(kernel_src: str, workload: str):
