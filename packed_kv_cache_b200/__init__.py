@@ -136,6 +136,17 @@ def _dev(t, name: str):
     return t.data_ptr()
 
 
+def _expect(t, name: str, dtype, min_numel: int) -> None:
+    """Refuse a tensor of the wrong element type, or with fewer elements than
+    the call reads or writes: the library sees only its address."""
+    if t is None or not isinstance(t, torch.Tensor):
+        return
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype} (got {t.dtype})")
+    if t.numel() < min_numel:
+        raise ValueError(f"{name} has {t.numel()} elements; the call needs at least {min_numel}")
+
+
 def _stream(stream) -> int | None:
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
@@ -275,17 +286,49 @@ class PackedKVCache:
     def info(self, layer: int) -> dict:
         return pf_cache_layer_info(self.handle, layer)
 
+    # sizes the calls read and write, from the configuration
+    def _rows(self, rows: int) -> int:
+        """Elements of a [B, rows, H, D] tensor."""
+        c = self.cfg
+        return c.batch * rows * c.heads * c.head_dim
+
+    def _n(self) -> int:
+        return self.cfg.block_frames * self.cfg.h * self.cfg.w
+
+    def _n_c(self) -> int:
+        c = self.cfg
+        return (c.block_frames // 2) * (c.h // 4) * (c.w // 4)
+
+    def _check_selection_buffers(self, layer, sel_out=None, scores_out=None, scores_in=None) -> None:
+        if sel_out is None and scores_out is None and scores_in is None:
+            return
+        live = self.info(layer)["mid_count"]
+        B = self.cfg.batch
+        _expect(sel_out, "sel_out", torch.int32, B * min(self.cfg.n_top, live))
+        _expect(scores_out, "scores_out", torch.float32, B * live)
+        _expect(scores_in, "scores_in", torch.float32, B * live)
+
     def append_block(self, layer, K, V, Kc=None, Vc=None, stream=None) -> int:
+        for t, name in ((K, "K"), (V, "V")):
+            _expect(t, name, torch.bfloat16, self._rows(self._n()))
+        for t, name in ((Kc, "Kc"), (Vc, "Vc")):
+            _expect(t, name, torch.bfloat16, self._rows(self._n_c()))
         return pf_cache_append_block(self.handle, layer, K, V, Kc, Vc, stream)
 
     def load_mid(self, layer, Kc, Vc, stream=None) -> int:
+        for t, name in ((Kc, "Kc"), (Vc, "Vc")):
+            _expect(t, name, torch.bfloat16, self._rows(self._n_c()) * Kc.shape[1])
         return pf_cache_load_mid(self.handle, layer, Kc, Vc, Kc.shape[1], stream)
 
     def select_mid(self, layer, Q, sel_out=None, scores_out=None, stream=None) -> None:
+        _expect(Q, "Q", torch.bfloat16, self._rows(self._n()))
+        self._check_selection_buffers(layer, sel_out, scores_out)
         pf_select_mid(self.handle, layer, Q, sel_out, scores_out, stream)
 
     def select_mid_ex(self, layer, Q=None, policy=ROUTE_SCORE, q_stride=1, heads=None, heads_total=0,
                       scores_in=None, sel_out=None, scores_out=None, stream=None) -> None:
+        _expect(Q, "Q", torch.bfloat16, self._rows(self._n()))
+        self._check_selection_buffers(layer, sel_out, scores_out, scores_in)
         pf_select_mid_ex(self.handle, layer, Q, policy, q_stride, heads, heads_total, scores_in, sel_out,
                          scores_out, stream)
 
@@ -293,6 +336,10 @@ class PackedKVCache:
         pf_rope_shift(self.handle, layer, parts, delta, stream)
 
     def attend(self, layer, Q, K_cur, V_cur, O=None, lse=None, stream=None) -> torch.Tensor:
+        need = self._rows(self._n())
+        for t, name in ((Q, "Q"), (K_cur, "K_cur"), (V_cur, "V_cur"), (O, "O")):
+            _expect(t, name, torch.bfloat16, need)
+        _expect(lse, "lse", torch.float32, need // self.cfg.head_dim)
         if O is None:
             O = torch.empty_like(Q)
         pf_attend(self.handle, layer, Q, K_cur, V_cur, O, lse, stream)

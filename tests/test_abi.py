@@ -157,6 +157,44 @@ def test_static_selection_checks_arguments_before_device_work(pf):
     assert call(count=0) == 0 and call(n_top=0) == 0
 
 
+def test_cache_methods_refuse_wrong_dtypes_and_short_buffers(pf):
+    # the library sees only addresses: the binding refuses a buffer of the wrong
+    # element type or too small for the call before anything is launched.
+    # (No GPU here: an object without an arena, with the layer's live-block
+    # count stubbed; a correct CPU tensor passes the checks and is then refused
+    # as not being on the device.)
+    import torch
+    wl = synth.WORKLOADS["ragged_a"]                  # B=2, H=2, n=240, n_c=4, n_top=5
+    cache = pf.PackedKVCache.__new__(pf.PackedKVCache)
+    cache.cfg, cache.handle = pf.config_for(wl), None
+    cache.info = lambda layer: {"mid_count": 13}
+    B, H, D, n, nc = wl.batch, wl.heads, wl.head_dim, wl.n, wl.n_c
+    bf = lambda *shape: torch.zeros(shape, dtype=torch.bfloat16)   # noqa: E731
+    Q = bf(B, n, H, D)
+
+    def refused(fn, what):
+        with pytest.raises(ValueError) as e:
+            fn()
+        assert what in str(e.value), str(e.value)
+
+    refused(lambda: cache.attend(0, Q.float(), Q, Q), "Q must be torch.bfloat16")
+    refused(lambda: cache.attend(0, Q, Q[:, :-1], Q), "K_cur has")
+    refused(lambda: cache.attend(0, Q, Q, Q, O=bf(B, n - 1, H, D)), "O has")
+    refused(lambda: cache.attend(0, Q, Q, Q, lse=torch.zeros(B * H * n - 1)), "lse has")
+    refused(lambda: cache.attend(0, Q, Q, Q), "CUDA tensor")
+    refused(lambda: cache.select_mid(0, bf(B, n, H, D - 1)), "Q has")
+    refused(lambda: cache.select_mid(0, Q, torch.zeros((B, 4), dtype=torch.int32)), "sel_out has")
+    refused(lambda: cache.select_mid(0, Q, torch.zeros((B, 5), dtype=torch.int64)), "sel_out must be")
+    refused(lambda: cache.select_mid(0, Q, None, torch.zeros((B, 12))), "scores_out has")
+    refused(lambda: cache.select_mid(0, Q, torch.zeros((B, 5), dtype=torch.int32), torch.zeros((B, 13))),
+            "CUDA tensor")
+    refused(lambda: cache.select_mid_ex(0, None, policy=pf.ROUTE_GIVEN, scores_in=torch.zeros((B, 12))),
+            "scores_in has")
+    refused(lambda: cache.append_block(0, Q[:, :-1], Q), "K has")
+    refused(lambda: cache.append_block(0, Q, Q, bf(B, nc - 1, H, D), bf(B, nc, H, D)), "Kc has")
+    refused(lambda: cache.load_mid(0, bf(B, 3, nc, H, D), bf(B, 2, nc, H, D)), "Vc has")
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     # importing the binding from a copy without libpf.so must raise, not fall back
     import shutil
