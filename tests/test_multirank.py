@@ -36,7 +36,7 @@ def _worker(rank, world, port, out):
 def test_two_gloo_ranks_max_time_and_distinct_seeds():
     world = 2
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
     assert out[0][0] == out[1][0] == 15.0
@@ -75,7 +75,7 @@ def _shard_worker(rank, world, port, out):
 def test_head_sharded_selection_exchange_on_two_gloo_ranks():
     world = 2
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_shard_worker, args=(world, port, out), nprocs=world, join=True)
     import numpy as np
