@@ -5,7 +5,6 @@ of each rank's heads, summed across ranks before the top-k)."""
 import os
 import socket
 
-import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
