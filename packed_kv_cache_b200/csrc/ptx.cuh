@@ -234,8 +234,9 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // 2^x on the FMA and integer pipes: x = n + f, n = round(x) (by adding and
 // subtracting 1.5 * 2^23), f in [-1/2, 1/2]; 2^f by a cubic fitted for the
 // least maximum relative error (7.5e-5; packed_kv_cache_b200/fit_exp2.py);
-// 2^n added to the exponent bits.  x is clamped below at -126, so results
-// are normal floats (the smallest is about 1.2e-38 instead of 0).
+// 2^n added to the exponent bits.  x is clamped below at -126, so the
+// smallest result is about 1.2e-38 instead of 0 (at the clamp the cubic is
+// just under 1 and the sum falls into the subnormal encoding: 1.17533e-38).
 __device__ __forceinline__ float ex2_poly(float x) {
   x = fmaxf(x, -126.0f);
   const float t = x + 12582912.0f;
