@@ -12,6 +12,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -82,6 +83,18 @@ pf_status check_config(const pf_config* c) {
   if (c->mid_capacity + c->recent_blocks > kMaxPoolSlots)
     return fail(PF_ERR_CAPACITY, "mid_capacity + recent_blocks must be <= %d", kMaxPoolSlots);
   if (1LL * c->heads * c->head_dim > 65536) return fail(PF_ERR_CAPACITY, "too many heads");
+  // The attention kernel walks the context in 32-key sub-boxes, counted in
+  // int, and finds a sub-box's block by a float-reciprocal quotient that is
+  // exact below 2^22 sub-boxes: the context, padded as the kernel pads it,
+  // stays below 2^27 keys.
+  const long long sub = 32;
+  const long long blk_keys = (n + sub - 1) / sub * sub;
+  const long long mid_keys = n_c > 0 ? (n_c + sub - 1) / sub * sub * std::min(c->n_top, c->mid_capacity) : 0;
+  const long long sink_keys = (c->sink_blocks * n + sub - 1) / sub * sub;
+  const long long context = sink_keys + mid_keys + (c->recent_blocks + 1LL) * blk_keys;
+  if (context >= (1LL << 27))
+    return fail(PF_ERR_CAPACITY, "attention context of %lld keys (in 32-key sub-boxes) must stay below 2^27",
+                context);
   return PF_OK;
 }
 

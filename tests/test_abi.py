@@ -87,9 +87,10 @@ def test_config_validation(pf, field, value, status):
 
 
 def test_cache_bytes_reports_overflow_instead_of_wrapping(pf):
-    # 2^31 batch items x 2^31 sink blocks x 2^24 tokens x 128 KB rows is far
-    # past size_t: the size must be refused, never wrapped to a small arena
-    big = dict(batch=2**31 - 1, sink_blocks=2**31 - 1, heads=512, block_frames=2, h=4096, w=2048)
+    # 2^31 layers of 2^31 batch items with 128 KB key rows (a pages-scale
+    # context of 28,032 keys) is far past size_t: the size must be refused,
+    # never wrapped to a small arena
+    big = dict(batch=2**31 - 1, layers=2**31 - 1, heads=512)
     with pytest.raises(pf.PFError) as e:
         pf.pf_cache_bytes(_cfg(pf, **big))
     assert e.value.status_name == "PF_ERR_CAPACITY"
@@ -100,6 +101,44 @@ def test_cache_bytes_reports_overflow_instead_of_wrapping(pf):
     # the largest sizes that still fit are computed exactly
     one, two = (pf.pf_cache_bytes(_cfg(pf, layers=k)) for k in (1, 2))
     assert pf.pf_cache_bytes(_cfg(pf, layers=2**31 - 1)) == one + (2**31 - 2) * (two - one)
+
+
+def test_attention_context_is_capped_below_2_27_keys(pf):
+    # n = 4 x 512 x 512 = 2^20 keys per block, one head; the context counted as
+    # the attention pads it: sink + routed mid blocks + recent + current
+    base = dict(heads=1, block_frames=4, h=512, w=512)
+
+    def status(**kw):
+        try:
+            pf.pf_cache_bytes(_cfg(pf, **dict(base, **kw)))
+            return "PF_OK"
+        except pf.PFError as e:
+            return e.status_name
+
+    none = dict(sink_blocks=0, mid_capacity=0, n_top=0)
+    assert status(recent_blocks=126, **none) == "PF_OK"              # 127 x 2^20 keys
+    assert status(recent_blocks=127, **none) == "PF_ERR_CAPACITY"    # 2^27 keys
+    assert b"2^27" in pf.lib.pf_last_error()
+    assert status(recent_blocks=1, sink_blocks=125, mid_capacity=0, n_top=0) == "PF_OK"
+    assert status(recent_blocks=1, sink_blocks=126, mid_capacity=0, n_top=0) == "PF_ERR_CAPACITY"
+    # routed mid blocks: min(n_top, mid_capacity) blocks of n_c = 2 x 128 x 128 = 2^15 keys
+    assert status(recent_blocks=126, sink_blocks=0, mid_capacity=31, n_top=1000) == "PF_OK"
+    assert status(recent_blocks=126, sink_blocks=0, mid_capacity=32, n_top=1000) == "PF_ERR_CAPACITY"
+    assert status(recent_blocks=126, sink_blocks=0, mid_capacity=1000, n_top=31) == "PF_OK"
+
+
+def test_every_configuration_the_tests_and_the_bench_build_is_accepted(pf):
+    W = synth.WORKLOADS
+    cases = list(W.values()) + [
+        W["tiny"].replace(mid_capacity=8191, pool_blocks=8191, planted=16, n_top=16),
+        W["tiny"].replace(mid_capacity=8191, pool_blocks=8191, planted=0, n_top=3000),
+        W["ragged_a"].replace(pool_blocks=9, planted=0, mid_capacity=9, n_top=4),
+        W["ragged_a"].replace(n_top=0, planted=0),
+        W["tiny"].replace(mid_capacity=3, recent_blocks=2, n_top=2, planted=0, pool_blocks=0),
+        W["ragged_a"].replace(mid_capacity=4, n_top=2, planted=0)]
+    for wl in cases:
+        for fused in (False, True):
+            assert pf.pf_cache_bytes(pf.config_for(wl, sink_rope_in_attention=fused)) > 0, wl.name
 
 
 def test_rope_split_validation(pf):

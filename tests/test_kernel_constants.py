@@ -1,9 +1,15 @@
-"""Host checks of constants compiled into the kernels: the cubic that the
-attention softmax can use for part of its exponentials (an option of the
-attention kernel).  The coefficients in ptx.cuh must be the ones the fitting
-script produces, and the whole evaluation (round-to-integer by the 1.5 * 2^23
-trick, cubic on the fraction, exponent bits added) must stay within the
-stated relative error.  CPU only."""
+"""Host checks of constants and arithmetic tricks compiled into the kernels,
+emulated in float32 with numpy.  CPU only.
+
+* The cubic that the attention softmax can use for part of its exponentials
+  (an option of the attention kernel): the coefficients in ptx.cuh must be
+  the ones the fitting script produces, and the whole evaluation (round to
+  integer by the 1.5 * 2^23 trick, cubic on the fraction, exponent bits
+  added) must stay within the stated relative error.
+* The attention producer's division by a run-time sub-box count (a float
+  reciprocal quotient corrected by one step): exact over every argument the
+  kernel can see, which the configuration check bounds (fewer than 2^22
+  sub-boxes per context, at most 8,192 pool or recent slots)."""
 import importlib.util
 import os
 import re
@@ -67,3 +73,40 @@ def test_evaluation_error_over_the_softmax_range():
     # is just under 1 there, so the encoding is subnormal): never 0, NaN or large
     low = _ex2_poly_f32(np.array([-126.0, -200.0, -1e4, -1e30]), c).astype(np.float64)
     assert np.all(low == low[0]) and abs(low[0] / 2.0 ** -126 - 1) < 2e-4
+
+
+def _div_small(a, b, inv_b):
+    """floor(a / b) the kernel's way: q = trunc(float(a) * inv_b) in float32,
+    then one correction step on the remainder."""
+    q = np.trunc(a.astype(np.float32) * np.float32(inv_b)).astype(np.int64)
+    r = a - q * b
+    return np.where(r < 0, q - 1, np.where(r >= b, q + 1, q))
+
+
+def _inverses(b):
+    # 1.f / b as compiled (IEEE division, correctly rounded), and one ulp either
+    # side, so that the result does not hang on the last bit of the reciprocal
+    inv = np.float32(1.0) / np.float32(b)
+    return [inv, np.nextafter(inv, np.float32(0)), np.nextafter(inv, np.float32(1))]
+
+
+def test_division_by_sub_box_counts_is_exact():
+    A_MAX, SLOTS = 1 << 22, 8192
+    # every numerator for small divisors (sub-boxes per compressed block: 6 at
+    # the pages' scale)
+    for b in range(1, 65):
+        a = np.arange(min(A_MAX, SLOTS * b), dtype=np.int64)
+        for inv in _inverses(b):
+            assert np.array_equal(_div_small(a, b, inv), a // b), b
+    # larger divisors (sub-boxes per full block: 195 at the pages' scale, up to
+    # 2^19): each quotient's first and last numerator, and its neighbours
+    rng = np.random.default_rng(0)
+    bs = sorted({65, 100, 127, 128, 129, 195, 390, 1000, 4093, 4096, 6240, 65521, 65536, 99991,
+                 (1 << 19) - 1, 1 << 19} | set(rng.integers(65, 1 << 19, 40).tolist()))
+    for b in bs:
+        q = np.arange(min(SLOTS, A_MAX // b + 1), dtype=np.int64)
+        a = np.concatenate([q * b, q * b + b - 1, q * b + 1, np.maximum(q * b - 1, 0),
+                            rng.integers(0, min(A_MAX, SLOTS * b), 4096)])
+        a = a[a < min(A_MAX, SLOTS * b)]
+        for inv in _inverses(b):
+            assert np.array_equal(_div_small(a, b, inv), a // b), b
