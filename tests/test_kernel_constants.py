@@ -9,7 +9,9 @@ emulated in float32 with numpy.  CPU only.
 * The attention producer's division by a run-time sub-box count (a float
   reciprocal quotient corrected by one step): exact over every argument the
   kernel can see, which the configuration check bounds (fewer than 2^22
-  sub-boxes per context, at most 8,192 pool or recent slots)."""
+  sub-boxes per context, at most 8,192 pool or recent slots).
+* The selection's radix top-k ranks float scores by an unsigned key: the key
+  order must be the float order, with -0 and +0 equal."""
 import importlib.util
 import os
 import re
@@ -110,3 +112,26 @@ def test_division_by_sub_box_counts_is_exact():
         a = a[a < min(A_MAX, SLOTS * b)]
         for inv in _inverses(b):
             assert np.array_equal(_div_small(a, b, inv), a // b), b
+
+
+def _order_key(f):
+    """The selection's key: -0 made +0, then negative floats bit-inverted and
+    non-negative ones given the top bit."""
+    u = (f.astype(np.float32) + np.float32(0.0)).view(np.uint32)
+    return np.where(u & np.uint32(0x80000000), ~u, u | np.uint32(0x80000000))
+
+
+def test_order_key_sorts_like_the_scores():
+    rng = np.random.default_rng(1)
+    tiny = np.finfo(np.float32).tiny
+    special = np.array([0.0, -0.0, tiny, -tiny, tiny / 8, -tiny / 8, 1.0, -1.0,
+                        np.finfo(np.float32).max, -np.finfo(np.float32).max, np.inf, -np.inf], dtype=np.float32)
+    f = np.concatenate([special, rng.standard_normal(20000).astype(np.float32),
+                        (rng.standard_normal(5000) * 1e-30).astype(np.float32),
+                        rng.integers(0, 2**32, 5000, dtype=np.uint64).astype(np.uint32).view(np.float32)])
+    f = f[~np.isnan(f)]
+    k = _order_key(f)
+    i, j = rng.integers(0, len(f), (2, 200000))
+    assert np.array_equal(f[i] < f[j], k[i] < k[j])
+    assert np.array_equal(f[i] == f[j], k[i] == k[j])             # -0 == +0 on both sides
+    assert _order_key(np.array([-0.0], np.float32))[0] == _order_key(np.array([0.0], np.float32))[0]
