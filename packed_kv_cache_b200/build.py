@@ -6,6 +6,8 @@ with PF_ERR_CUDA).  Usage:  python -m packed_kv_cache_b200.build [--verbose]
 """
 from __future__ import annotations
 
+import contextlib
+import fcntl
 import os
 import subprocess
 import sys
@@ -17,6 +19,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libpf.so")
+LOCK = os.path.join(HERE, ".build.lock")
 
 SOURCES = ["pf_cache.cpp", "rope_shift.cu", "append_copy.cu", "select.cu", "attend.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -55,19 +58,35 @@ def _stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
+@contextlib.contextmanager
+def _exclusive():
+    """One build at a time across processes: the ranks of one job, or parallel
+    test workers, may all find the library stale and would otherwise write the
+    same object files at once."""
+    with open(LOCK, "a") as f:
+        fcntl.flock(f, fcntl.LOCK_EX)
+        try:
+            yield
+        finally:
+            fcntl.flock(f, fcntl.LOCK_UN)
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     """Compile and link libpf.so if any source is newer than it; return its path."""
     if not force and not _stale():
         return LIB
-    os.makedirs(BUILD, exist_ok=True)
-    with ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose), SOURCES))
-    tmp = LIB + ".tmp"
-    cmd = [nvcc(), "-shared", "-o", tmp] + objs + ARCH + ["-cudart", "static", "-Xcompiler", "-fPIC"]
-    r = subprocess.run(cmd, capture_output=True, text=True)
-    if r.returncode != 0:
-        raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
+    with _exclusive():
+        if not force and not _stale():   # built by another process while this one waited
+            return LIB
+        os.makedirs(BUILD, exist_ok=True)
+        with ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
+            objs = list(ex.map(lambda s: _compile(s, verbose), SOURCES))
+        tmp = f"{LIB}.{os.getpid()}.tmp"
+        cmd = [nvcc(), "-shared", "-o", tmp] + objs + ARCH + ["-cudart", "static", "-Xcompiler", "-fPIC"]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0:
+            raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
+        os.replace(tmp, LIB)
     return LIB
 
 

@@ -234,6 +234,35 @@ def test_cache_methods_refuse_wrong_dtypes_and_short_buffers(pf):
     refused(lambda: cache.load_mid(0, bf(B, 3, nc, H, D), bf(B, 2, nc, H, D)), "Vc has")
 
 
+def _hold_build_lock(q):
+    import time
+
+    from packed_kv_cache_b200 import build
+    with build._exclusive():
+        t0 = time.monotonic()
+        time.sleep(0.3)
+        q.put((t0, time.monotonic()))
+
+
+def test_builds_in_several_processes_take_turns(pf):
+    # the ranks of one job may all find the library stale: the build lock lets
+    # one process compile at a time (the others then find it fresh)
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_hold_build_lock, args=(q,)) for _ in range(3)]
+    for p in procs:
+        p.start()
+    spans = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for (a0, a1), (b0, b1) in zip(spans, spans[1:]):
+        assert a1 <= b0, spans                       # no two holders at once
+    from packed_kv_cache_b200 import build
+    assert build.build() == build.LIB                # fresh: returns without taking the lock
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     # importing the binding from a copy without libpf.so must raise, not fall back
     import shutil
