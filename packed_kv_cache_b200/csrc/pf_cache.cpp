@@ -75,12 +75,13 @@ pf_status check_config(const pf_config* c) {
   if (!(c->rope_base > 1.0f)) return fail(PF_ERR_ARG, "rope_base must be > 1");
   if (c->sink_rope_in_attention != 0 && c->sink_rope_in_attention != 1)
     return fail(PF_ERR_ARG, "sink_rope_in_attention must be 0 or 1");
-  const long long n = 1LL * c->block_frames * c->h * c->w;
-  if (n > (1 << 24)) return fail(PF_ERR_CAPACITY, "block of %lld tokens is too large", n);
+  long long n = 1LL * c->block_frames * c->h;  // both positive ints: no overflow
+  if (n <= (1 << 24)) n *= c->w;                 // nor here
+  if (n > (1 << 24)) return fail(PF_ERR_CAPACITY, "a block holds at most 2^24 tokens (B_f * h * w)");
   const long long n_c = 1LL * (c->block_frames / 2) * (c->h / 4) * (c->w / 4);
   if (n_c <= 0 && c->mid_capacity > 0)
     return fail(PF_ERR_ARG, "compressed blocks would be empty (B_f >= 2, h >= 4, w >= 4 needed)");
-  if (c->mid_capacity + c->recent_blocks > kMaxPoolSlots)
+  if (1LL * c->mid_capacity + c->recent_blocks > kMaxPoolSlots)
     return fail(PF_ERR_CAPACITY, "mid_capacity + recent_blocks must be <= %d", kMaxPoolSlots);
   if (1LL * c->heads * c->head_dim > 65536) return fail(PF_ERR_CAPACITY, "too many heads");
   // The attention kernel walks the context in 32-key sub-boxes, counted in

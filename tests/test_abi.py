@@ -78,6 +78,9 @@ def test_cache_bytes_layout(pf):
     ("recent_blocks", 0, "PF_ERR_ARG"),
     ("mid_capacity", 9000, "PF_ERR_CAPACITY"),
     ("rope_base", 0.5, "PF_ERR_ARG"),
+    # sums and products of int fields that would overflow if formed in int
+    ("mid_capacity", 2**31 - 1, "PF_ERR_CAPACITY"),
+    ("h", 2**31 - 1, "PF_ERR_CAPACITY"),
 ])
 def test_config_validation(pf, field, value, status):
     c = _cfg(pf, **{field: value})
@@ -139,6 +142,16 @@ def test_every_configuration_the_tests_and_the_bench_build_is_accepted(pf):
     for wl in cases:
         for fused in (False, True):
             assert pf.pf_cache_bytes(pf.config_for(wl, sink_rope_in_attention=fused)) > 0, wl.name
+
+
+def test_block_size_product_does_not_overflow(pf):
+    # B_f * h * w with every factor near 2^31 overflows even 64 bits when
+    # formed in one go; the check refuses it instead
+    for kw in (dict(block_frames=2**31 - 1, h=2**31 - 1, w=2**31 - 1), dict(block_frames=4, h=2**30, w=2**30),
+               dict(block_frames=2**31 - 1, h=1, w=1)):
+        with pytest.raises(pf.PFError) as e:
+            pf.pf_cache_bytes(_cfg(pf, **kw))
+        assert e.value.status_name == "PF_ERR_CAPACITY" and b"2^24" in pf.lib.pf_last_error()
 
 
 def test_rope_split_validation(pf):
