@@ -276,6 +276,44 @@ def test_builds_in_several_processes_take_turns(pf):
     assert build.build() == build.LIB                # fresh: returns without taking the lock
 
 
+def test_binding_structs_and_constants_match_the_header(pf, tmp_path):
+    # every ctypes struct field at the offset the C compiler gives it, the same
+    # sizes, and the same numeric constants (a mismatch would corrupt every call)
+    import shutil
+    import subprocess
+    if not shutil.which("gcc"):
+        pytest.skip("needs gcc")
+    structs = {"pf_config": pf.Config, "pf_select_opts": pf.SelectOpts, "pf_layer_info": pf.LayerInfo}
+    lines = ["#include <stddef.h>", "#include <stdio.h>", '#include "pf.h"', "int main(void) {"]
+    for cname, cls in structs.items():
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for field, _ in cls._fields_:
+            lines.append(f'  printf("{cname} {field} %zu\\n", offsetof({cname}, {field}));')
+    consts = ["PF_PART_SINK", "PF_PART_MID", "PF_PART_RECENT", "PF_ROUTE_SCORE", "PF_ROUTE_SCORES_ONLY",
+              "PF_ROUTE_GIVEN", "PF_ROUTE_FIFO"] + list(pf.STATUS.values())
+    for name in consts:
+        lines.append(f'  printf("const {name} %d\\n", (int)({name}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.splitlines():
+        a, b, v = line.split()
+        got[(a, b)] = int(v)
+    for cname, cls in structs.items():
+        assert got[(cname, "size")] == ctypes.sizeof(cls), cname
+        for field, _ in cls._fields_:
+            assert got[(cname, field)] == getattr(cls, field).offset, (cname, field)
+    py = {"PF_PART_SINK": pf.PART_SINK, "PF_PART_MID": pf.PART_MID, "PF_PART_RECENT": pf.PART_RECENT,
+          "PF_ROUTE_SCORE": pf.ROUTE_SCORE, "PF_ROUTE_SCORES_ONLY": pf.ROUTE_SCORES_ONLY,
+          "PF_ROUTE_GIVEN": pf.ROUTE_GIVEN, "PF_ROUTE_FIFO": pf.ROUTE_FIFO}
+    py.update({name: code for code, name in pf.STATUS.items()})
+    for name in consts:
+        assert got[("const", name)] == py[name], name
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     # importing the binding from a copy without libpf.so must raise, not fall back
     import shutil
