@@ -314,6 +314,37 @@ def test_binding_structs_and_constants_match_the_header(pf, tmp_path):
         assert got[("const", name)] == py[name], name
 
 
+def _c_kind(decl: str) -> str:
+    decl = decl.strip()
+    if "*" in decl:
+        return "pointer"
+    words = decl.replace("const", "").split()
+    base = " ".join(words[:-1]) if len(words) > 1 else words[0]
+    return {"int": "int", "pf_status": "int", "unsigned": "unsigned", "unsigned int": "unsigned",
+            "size_t": "size_t", "float": "float"}[base]
+
+
+def _ctypes_kind(t) -> str:
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or hasattr(t, "_type_") and isinstance(t._type_, type):
+        return "pointer"
+    return {ctypes.c_int: "int", ctypes.c_uint: "unsigned", ctypes.c_size_t: "size_t",
+            ctypes.c_float: "float"}[t]
+
+
+def test_binding_argtypes_match_the_prototypes(pf):
+    # each declared function: the same number of parameters, each of the same
+    # kind (pointer, int, unsigned, size_t, float), and the same result kind
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    protos = re.findall(r"([A-Za-z_][\w ]*?\**)\s*\b(pf_[a-z_0-9]+)\s*\(([^)]*)\)\s*;", text)
+    assert len(protos) == len(declared_functions())
+    for ret, name, params in protos:
+        f = getattr(pf.lib, name)
+        assert f.argtypes is not None, name
+        kinds = [] if params.strip() in ("", "void") else [_c_kind(p) for p in params.split(",")]
+        assert kinds == [_ctypes_kind(t) for t in f.argtypes], name
+        assert _c_kind(ret + " r") == _ctypes_kind(f.restype), name
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     # importing the binding from a copy without libpf.so must raise, not fall back
     import shutil
