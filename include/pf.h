@@ -216,7 +216,7 @@ pf_status pf_select_mid(pf_cache* cache, int layer, const void* Q, int32_t* sel_
 
 typedef struct pf_select_opts {
   int policy;             /* PF_ROUTE_* */
-  int q_stride;           /* >= 1; 1 = every query row */
+  int q_stride;           /* >= 1; 1 = every query row; >= n: row 0 only */
   int head_lo, head_hi;   /* heads used by the score; head_hi = 0 means all */
   int heads_total;        /* score divisor in heads; 0 = the heads used */
   const float* scores_in; /* PF_ROUTE_GIVEN only */

@@ -562,6 +562,7 @@ pf_status pf_select_mid_ex(pf_cache* c, int layer, const void* Q, const pf_selec
   if (o.head_lo == 0 && o.head_hi == 0) o.head_hi = cf.heads;
   if (o.policy < PF_ROUTE_SCORE || o.policy > PF_ROUTE_FIFO) return fail(PF_ERR_ARG, "unknown routing policy %d", o.policy);
   if (o.q_stride < 1) return fail(PF_ERR_ARG, "q_stride %d < 1", o.q_stride);
+  if (o.q_stride > g.n) o.q_stride = g.n;  // the same rows (row 0 only); keeps n + q_stride in int
   if (o.head_lo < 0 || o.head_hi > cf.heads || o.head_lo >= o.head_hi)
     return fail(PF_ERR_ARG, "head range [%d, %d) not inside [0, %d)", o.head_lo, o.head_hi, cf.heads);
   if (o.heads_total < 0) return fail(PF_ERR_ARG, "heads_total %d < 0", o.heads_total);
