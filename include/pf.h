@@ -116,7 +116,7 @@ const char* pf_status_string(pf_status s);
  * Errors: PF_ERR_ARG for a null pointer or a non-positive size,
  * PF_ERR_UNSUPPORTED for head_dim != 128 or rope_split not summing to it,
  * PF_ERR_CAPACITY when a size limit is exceeded or the total does not fit
- * in size_t.  Limits: a block of at most 2^24 tokens, H * D <= 65536,
+ * in size_t.  Limits: a block of at most 2^24 tokens, H * D <= 32768,
  * mid_capacity + recent_blocks <= 8192, and an attention context (sink +
  * min(n_top, mid_capacity) compressed blocks + recent + current, each
  * partition rounded up to 32 keys) below 2^27 keys.

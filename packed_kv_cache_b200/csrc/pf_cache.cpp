@@ -83,7 +83,9 @@ pf_status check_config(const pf_config* c) {
     return fail(PF_ERR_ARG, "compressed blocks would be empty (B_f >= 2, h >= 4, w >= 4 needed)");
   if (1LL * c->mid_capacity + c->recent_blocks > kMaxPoolSlots)
     return fail(PF_ERR_CAPACITY, "mid_capacity + recent_blocks must be <= %d", kMaxPoolSlots);
-  if (1LL * c->heads * c->head_dim > 65536) return fail(PF_ERR_CAPACITY, "too many heads");
+  // the scoring kernel keeps the pooled query (H * D floats) and every pool
+  // score (kMaxPoolSlots keys) in shared memory: 128 KB + 32 KB at most
+  if (1LL * c->heads * c->head_dim > 32768) return fail(PF_ERR_CAPACITY, "H * D must be <= 32768 (at most 256 heads)");
   // The attention kernel walks the context in 32-key sub-boxes, counted in
   // int, and finds a sub-box's block by a float-reciprocal quotient that is
   // exact below 2^22 sub-boxes: the context, padded as the kernel pads it,

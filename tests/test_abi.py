@@ -81,6 +81,7 @@ def test_cache_bytes_layout(pf):
     # sums and products of int fields that would overflow if formed in int
     ("mid_capacity", 2**31 - 1, "PF_ERR_CAPACITY"),
     ("h", 2**31 - 1, "PF_ERR_CAPACITY"),
+    ("heads", 257, "PF_ERR_CAPACITY"),     # the scoring kernel's shared memory
 ])
 def test_config_validation(pf, field, value, status):
     c = _cfg(pf, **{field: value})
@@ -90,10 +91,10 @@ def test_config_validation(pf, field, value, status):
 
 
 def test_cache_bytes_reports_overflow_instead_of_wrapping(pf):
-    # 2^31 layers of 2^31 batch items with 128 KB key rows (a pages-scale
+    # 2^31 layers of 2^31 batch items with 64 KB key rows (a pages-scale
     # context of 28,032 keys) is far past size_t: the size must be refused,
     # never wrapped to a small arena
-    big = dict(batch=2**31 - 1, layers=2**31 - 1, heads=512)
+    big = dict(batch=2**31 - 1, layers=2**31 - 1, heads=256)
     with pytest.raises(pf.PFError) as e:
         pf.pf_cache_bytes(_cfg(pf, **big))
     assert e.value.status_name == "PF_ERR_CAPACITY"
