@@ -36,6 +36,9 @@ STATUS = {0: "PF_OK", 1: "PF_ERR_ARG", 2: "PF_ERR_ARENA", 3: "PF_ERR_STATE", 4: 
 
 
 class PFError(RuntimeError):
+    """A library call returned a status other than PF_OK; carries the status
+    code, its name and the library's message for the calling thread."""
+
     def __init__(self, func: str, status: int, message: str):
         self.status = status
         self.status_name = STATUS.get(status, str(status))
@@ -43,6 +46,8 @@ class PFError(RuntimeError):
 
 
 class Config(ctypes.Structure):
+    """pf_config: the cache's shape (layers, batch, heads, block geometry,
+    partition sizes, routed count, rotary split and base)."""
     _fields_ = [("layers", ctypes.c_int), ("batch", ctypes.c_int), ("heads", ctypes.c_int),
                 ("head_dim", ctypes.c_int), ("block_frames", ctypes.c_int), ("h", ctypes.c_int),
                 ("w", ctypes.c_int), ("sink_blocks", ctypes.c_int), ("recent_blocks", ctypes.c_int),
@@ -52,11 +57,14 @@ class Config(ctypes.Structure):
 
 
 class SelectOpts(ctypes.Structure):
+    """pf_select_opts: routing policy, query stride, head range, score divisor."""
     _fields_ = [("policy", ctypes.c_int), ("q_stride", ctypes.c_int), ("head_lo", ctypes.c_int),
                 ("head_hi", ctypes.c_int), ("heads_total", ctypes.c_int), ("scores_in", ctypes.c_void_p)]
 
 
 class LayerInfo(ctypes.Structure):
+    """pf_layer_info: one layer's ring state and the device addresses of its
+    partitions."""
     _fields_ = [("blocks_seen", ctypes.c_int), ("sink_filled", ctypes.c_int),
                 ("recent_count", ctypes.c_int), ("recent_head", ctypes.c_int),
                 ("mid_count", ctypes.c_int), ("mid_head", ctypes.c_int), ("pool_slots", ctypes.c_int),
@@ -69,6 +77,7 @@ class LayerInfo(ctypes.Structure):
                 ("selection", ctypes.c_void_p), ("scores", ctypes.c_void_p)]
 
     def as_dict(self) -> dict:
+        """The fields by name."""
         return {name: getattr(self, name) for name, _ in self._fields_}
 
 
@@ -172,16 +181,21 @@ def config_for(wl, layers: int | None = None, sink_rope_in_attention: bool = Fal
 # ---------------------------------------------------------------- C-named calls
 
 def pf_version() -> int:
+    """Library version (100 = 0.1.0)."""
     return lib.pf_version()
 
 
 def pf_cache_bytes(cfg: Config) -> int:
+    """Arena bytes a cache of this configuration needs (token counts as in
+    PackForcing (arXiv), "KV Caching" and "Compressed Mid Tokens")."""
     out = ctypes.c_size_t()
     _check("pf_cache_bytes", lib.pf_cache_bytes(ctypes.byref(cfg), ctypes.byref(out)))
     return out.value
 
 
 def pf_cache_create(cfg: Config, arena, arena_bytes: int | None = None, stream=None) -> ctypes.c_void_p:
+    """A cache over a caller-owned, 256-byte aligned device arena (zeroed on
+    `stream`); returns the handle."""
     ptr = _dev(arena, "arena")
     nbytes = arena_bytes if arena_bytes is not None else arena.numel() * arena.element_size()
     handle = ctypes.c_void_p()
@@ -191,16 +205,21 @@ def pf_cache_create(cfg: Config, arena, arena_bytes: int | None = None, stream=N
 
 
 def pf_cache_destroy(handle) -> None:
+    """Free the cache's host state (the arena stays the caller's)."""
     _check("pf_cache_destroy", lib.pf_cache_destroy(handle))
 
 
 def pf_cache_layer_info(handle, layer: int) -> dict:
+    """Snapshot of one layer's state as a dict (LayerInfo fields)."""
     info = LayerInfo()
     _check("pf_cache_layer_info", lib.pf_cache_layer_info(handle, layer, ctypes.byref(info)))
     return info.as_dict()
 
 
 def pf_cache_append_block(handle, layer, K, V, Kc=None, Vc=None, stream=None) -> int:
+    """Append the finished block (PackForcing (arXiv), "Dual-Resolution
+    Shifting Mechanism"): sink until full, then recent, its compressed copy
+    joining the mid pool when it leaves; returns the blocks evicted (0 or 1)."""
     ev = ctypes.c_int(0)
     _check("pf_cache_append_block", lib.pf_cache_append_block(
         handle, layer, _dev(K, "K"), _dev(V, "V"), _dev(Kc, "Kc"), _dev(Vc, "Vc"), ctypes.byref(ev),
@@ -209,6 +228,8 @@ def pf_cache_append_block(handle, layer, K, V, Kc=None, Vc=None, stream=None) ->
 
 
 def pf_cache_load_mid(handle, layer, Kc, Vc, nblocks: int, stream=None) -> int:
+    """Push `nblocks` compressed blocks straight into the mid pool, oldest
+    first; returns the blocks evicted."""
     ev = ctypes.c_int(0)
     _check("pf_cache_load_mid", lib.pf_cache_load_mid(handle, layer, _dev(Kc, "Kc"), _dev(Vc, "Vc"),
                                                       nblocks, ctypes.byref(ev), _stream(stream)))
@@ -216,6 +237,9 @@ def pf_cache_load_mid(handle, layer, Kc, Vc, nblocks: int, stream=None) -> int:
 
 
 def pf_select_mid(handle, layer, Q, sel_out=None, scores_out=None, stream=None) -> None:
+    """Dynamic context selection (PackForcing digest, method step (3)): score
+    every live compressed block against the block's queries, keep the n_top
+    best (ties to the older block) for the layer's attention."""
     _check("pf_select_mid", lib.pf_select_mid(handle, layer, _dev(Q, "Q"), _dev(sel_out, "sel_out"),
                                               _dev(scores_out, "scores_out"), _stream(stream)))
 
@@ -234,21 +258,31 @@ def pf_select_mid_ex(handle, layer, Q, policy=ROUTE_SCORE, q_stride=1, heads=Non
 
 
 def pf_rope_shift(handle, layer: int, parts: int, delta: int, stream=None) -> None:
+    """Incremental temporal RoPE adjustment (PackForcing (arXiv), "Incremental
+    RoPE adjustment"): rotate the temporal pairs of the keys in `parts` by
+    delta frames, in place; layer -1 = every layer."""
     _check("pf_rope_shift", lib.pf_rope_shift(handle, layer, parts, delta, _stream(stream)))
 
 
 def pf_attend(handle, layer, Q, K_cur, V_cur, O, lse=None, stream=None) -> None:
+    """softmax(Q K^T / sqrt(d_h)) V over sink || selected mid || recent ||
+    current (PackForcing digest, KV-cache paragraph; PackForcing (arXiv),
+    "Bounded Attention Context"), into O; optional natural-log LSE."""
     _check("pf_attend", lib.pf_attend(handle, layer, _dev(Q, "Q"), _dev(K_cur, "K_cur"), _dev(V_cur, "V_cur"),
                                       _dev(O, "O"), _dev(lse, "lse"), _stream(stream)))
 
 
 def pf_poll_device_error(handle, stream=None) -> int:
+    """Synchronise `stream` and read (then clear) the cache's device error
+    word; raises PF_ERR_TIMEOUT if a bounded wait gave up."""
     code = ctypes.c_uint(0)
     _check("pf_poll_device_error", lib.pf_poll_device_error(handle, _stream(stream), ctypes.byref(code)))
     return code.value
 
 
 def pf_selftest_wait_timeout(handle, timeout_us: int, stream=None) -> None:
+    """Launch a kernel whose bounded wait on a flag nothing sets must give up
+    and report it (the failure-detection path, with no GPU fault)."""
     _check("pf_selftest_wait_timeout", lib.pf_selftest_wait_timeout(handle, timeout_us, _stream(stream)))
 
 
@@ -273,6 +307,7 @@ class PackedKVCache:
         self.handle = pf_cache_create(cfg, self.arena, self.nbytes, stream)
 
     def close(self) -> None:
+        """Free the host state; the arena tensor is released with the object."""
         if getattr(self, "handle", None):
             pf_cache_destroy(self.handle)
             self.handle = None
@@ -284,6 +319,7 @@ class PackedKVCache:
             pass
 
     def info(self, layer: int) -> dict:
+        """One layer's state (pf_cache_layer_info)."""
         return pf_cache_layer_info(self.handle, layer)
 
     # sizes the calls read and write, from the configuration
@@ -309,6 +345,8 @@ class PackedKVCache:
         _expect(scores_in, "scores_in", torch.float32, B * live)
 
     def append_block(self, layer, K, V, Kc=None, Vc=None, stream=None) -> int:
+        """K, V [B, n, H, 128] bf16; Kc, Vc [B, n_c, H, 128] bf16 (see
+        pf_cache_append_block).  Returns the blocks evicted."""
         for t, name in ((K, "K"), (V, "V")):
             _expect(t, name, torch.bfloat16, self._rows(self._n()))
         for t, name in ((Kc, "Kc"), (Vc, "Vc")):
@@ -316,26 +354,33 @@ class PackedKVCache:
         return pf_cache_append_block(self.handle, layer, K, V, Kc, Vc, stream)
 
     def load_mid(self, layer, Kc, Vc, stream=None) -> int:
+        """Kc, Vc [B, nblocks, n_c, H, 128] bf16 into the pool (see pf_cache_load_mid)."""
         for t, name in ((Kc, "Kc"), (Vc, "Vc")):
             _expect(t, name, torch.bfloat16, self._rows(self._n_c()) * Kc.shape[1])
         return pf_cache_load_mid(self.handle, layer, Kc, Vc, Kc.shape[1], stream)
 
     def select_mid(self, layer, Q, sel_out=None, scores_out=None, stream=None) -> None:
+        """Q [B, n, H, 128] bf16; optional sel_out [B, min(n_top, live)] int32
+        and scores_out [B, live] float32 (see pf_select_mid)."""
         _expect(Q, "Q", torch.bfloat16, self._rows(self._n()))
         self._check_selection_buffers(layer, sel_out, scores_out)
         pf_select_mid(self.handle, layer, Q, sel_out, scores_out, stream)
 
     def select_mid_ex(self, layer, Q=None, policy=ROUTE_SCORE, q_stride=1, heads=None, heads_total=0,
                       scores_in=None, sel_out=None, scores_out=None, stream=None) -> None:
+        """Selection with a routing policy (see pf_select_mid_ex)."""
         _expect(Q, "Q", torch.bfloat16, self._rows(self._n()))
         self._check_selection_buffers(layer, sel_out, scores_out, scores_in)
         pf_select_mid_ex(self.handle, layer, Q, policy, q_stride, heads, heads_total, scores_in, sel_out,
                          scores_out, stream)
 
     def rope_shift(self, layer, parts, delta, stream=None) -> None:
+        """Shift the keys of `parts` (PART_* mask) by delta frames (see pf_rope_shift)."""
         pf_rope_shift(self.handle, layer, parts, delta, stream)
 
     def attend(self, layer, Q, K_cur, V_cur, O=None, lse=None, stream=None) -> torch.Tensor:
+        """Q, K_cur, V_cur [B, n, H, 128] bf16 -> O (allocated if None); optional
+        lse [B, H, n] float32 (see pf_attend)."""
         need = self._rows(self._n())
         for t, name in ((Q, "Q"), (K_cur, "K_cur"), (V_cur, "V_cur"), (O, "O")):
             _expect(t, name, torch.bfloat16, need)
@@ -346,4 +391,5 @@ class PackedKVCache:
         return O
 
     def poll_device_error(self, stream=None) -> int:
+        """See pf_poll_device_error."""
         return pf_poll_device_error(self.handle, stream)
