@@ -28,6 +28,9 @@
  *    last message.  A failed call leaves the cache state unchanged.
  *  - Device-side failures (a bounded wait that gave up) are recorded in a
  *    word in the arena; pf_poll_device_error reads and clears it.
+ *  - One device per process: the attention kernel's shared-memory limit is
+ *    raised on the first device that launches it, so a second device in the
+ *    same process gets PF_ERR_CUDA from pf_attend.
  */
 #ifndef PF_H
 #define PF_H
