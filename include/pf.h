@@ -29,8 +29,8 @@
  *  - Device-side failures (a bounded wait that gave up) are recorded in a
  *    word in the arena; pf_poll_device_error reads and clears it.
  *  - One device per process: the attention kernel's shared-memory limit is
- *    raised on the first device that launches it, so a second device in the
- *    same process gets PF_ERR_CUDA from pf_attend.
+ *    raised once, on the first device that launches it; a second device in
+ *    the same process may get PF_ERR_CUDA from pf_attend.
  */
 #ifndef PF_H
 #define PF_H
