@@ -425,6 +425,18 @@ def oracle_step(d, wl, rows, heads=None):
     return attention_flops(B, H, len(rows), Lk, D)
 
 
+def cpu_model() -> str | None:
+    """The host CPU's model name (Linux), recorded beside the oracle's timing."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def cpu_baseline(d, wl, budget_s=15.0):
     import numpy as np
     dc = {k: (v.cpu() if hasattr(v, "cpu") else v) for k, v in d.items()}
@@ -443,7 +455,7 @@ def cpu_baseline(d, wl, budget_s=15.0):
     t0 = time.perf_counter()
     fl = oracle_step(dc, wl, rows)
     dt = time.perf_counter() - t0
-    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(), "cpu": cpu_model(), "kind": "oracle",
             "sample": (f"selection over the whole 40-block pool, sink RoPE shift, and attention of "
                        f"{nrows} of 6240 query rows x 12 heads over the 27872-key context, float64 numpy; "
                        f"{dt:.1f} s"), "seconds": round(dt, 2)}
@@ -506,7 +518,7 @@ def run_reference(args):
         "config": {"workload": ("one layer, pages scale: B=1, H=12, d_h=128, n=6240, pool 40x182, "
                                 "top-16, context 27872 keys; oracle sample per step"),
                    "rows_per_step": int(nr), "heads_per_step": int(nh)},
-        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": os.cpu_count(), "cpu": cpu_model(), "kind": "oracle",
                          "sample": f"per step, on {nh} of {wl.heads} heads: selection over the whole pool, "
                                    f"sink shift, attention of {nr} of {wl.n} query rows over the "
                                    f"27872-key context; float64 numpy"},
