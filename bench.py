@@ -386,7 +386,7 @@ def run_gpu(args):
         "gpu_launches": launches,
         "clocks": clk,
     }
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:   # the oracle's timing: one process only
         line["cpu_baseline"] = cpu_baseline(d, wl, budget_s=args.cpu_seconds)
     cache.close()
     if rank == 0:
