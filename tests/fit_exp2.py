@@ -7,7 +7,7 @@ error on [-1/2, 1/2] (Remez exchange on the relative error, started from
 Chebyshev nodes).  The result feeds a bf16 probability (8 significant bits),
 so a relative error near 1e-4 is far below its rounding.
 
-Run:  python packed_kv_cache_b200/fit_exp2.py
+Run:  python tests/fit_exp2.py
 """
 import numpy as np
 

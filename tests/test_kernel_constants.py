@@ -23,7 +23,7 @@ PTX = os.path.join(ROOT, "packed_kv_cache_b200", "csrc", "ptx.cuh")
 
 
 def _fit():
-    spec = importlib.util.spec_from_file_location("fit_exp2", os.path.join(ROOT, "packed_kv_cache_b200", "fit_exp2.py"))
+    spec = importlib.util.spec_from_file_location("fit_exp2", os.path.join(ROOT, "tests", "fit_exp2.py"))
     mod = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(mod)
     return mod.remez_relative()
