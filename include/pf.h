@@ -28,9 +28,12 @@
  *    last message.  A failed call leaves the cache state unchanged.
  *  - Device-side failures (a bounded wait that gave up) are recorded in a
  *    word in the arena; pf_poll_device_error reads and clears it.
- *  - One device per process: the attention kernel's shared-memory limit is
- *    raised once, on the first device that launches it; a second device in
- *    the same process may get PF_ERR_CUDA from pf_attend.
+ *  - Several devices (and host threads) may share the library: each
+ *    launcher's one-time set-up (a kernel attribute, a grid size) is done
+ *    once per device under a lock.  That set-up, and the address of the
+ *    allocation-free selection's array, belong to the device's primary
+ *    context: after cudaDeviceReset on a device the library must not be
+ *    used on it again in the same process.
  */
 #ifndef PF_H
 #define PF_H
@@ -276,6 +279,37 @@ pf_status pf_attend(pf_cache* cache, int layer, const void* Q, const void* K_cur
                     const void* V_cur, void* O, float* lse, void* stream);
 
 /*
+ * One layer's attention at one denoising step of the current block
+ * (PackForcing (arXiv), "Implementation Details": each block is denoised in
+ * S steps; digest, limitations paragraph: the context selection runs at a
+ * block's first denoising step only).  step == 0: pf_select_mid with this
+ * step's queries, then pf_attend; step > 0: pf_attend with the selection
+ * stored at step 0 (PF_ERR_STATE if the pool changed since, or if no
+ * selection was made while the pool holds more than n_top blocks).
+ * Arguments as for pf_attend; step >= 0.  Two or three kernel launches at
+ * step 0, one after.
+ */
+pf_status pf_attend_step(pf_cache* cache, int layer, int step, const void* Q, const void* K_cur,
+                         const void* V_cur, void* O, float* lse, void* stream);
+
+/*
+ * The current block is final (its last denoising step is done): append it
+ * to every layer and close the position gap of any eviction (PackForcing
+ * (arXiv), "Dual-Resolution Shifting Mechanism", "Incremental RoPE
+ * adjustment").  K, V, Kc, Vc: host arrays of `layers` device pointers, one
+ * per layer, each as for pf_cache_append_block.  Every layer's cache moves
+ * through the same states, so all layers evict together; if they evict,
+ * every layer's sink is shifted by evicted * B_f frames (pf_rope_shift,
+ * layer -1, PF_PART_SINK).  *evicted (optional) receives the blocks
+ * evicted per layer (0 or 1).  Every pointer is checked before anything is
+ * launched (PF_ERR_ARG leaves the cache unchanged); a launch failure
+ * (PF_ERR_CUDA) part-way leaves the layers before the failing one appended.
+ * Two launches per layer, plus one per layer for the shift.
+ */
+pf_status pf_finish_block(pf_cache* cache, const void* const* K, const void* const* V,
+                          const void* const* Kc, const void* const* Vc, int* evicted, void* stream);
+
+/*
  * Limits of pf_select_mid_static (its scratch is a fixed array in the library).
  */
 #define PF_STATIC_MAX_BATCH 8
@@ -301,13 +335,17 @@ pf_status pf_attend(pf_cache* cache, int layer, const void* Q, const void* K_cur
  *          compressed keys; the live blocks, oldest first, are the slots
  *          head, head+1, ... (mod pool_slots), `count` of them.
  * sel_out: [batch, min(n_top, count)] int32, device: the chosen blocks by
- *          age (0 = oldest live block), ascending.  Required.
- * scores_out (optional): [batch, count] float, device: the block scores.
+ *          age (0 = oldest live block), ascending.  Required (nothing is
+ *          written to it when n_top == 0).
+ * scores_out (optional): [batch, count] float, device: the block scores
+ *          (written for every n_top, 0 included).
  * Limits: batch <= PF_STATIC_MAX_BATCH, heads <= PF_STATIC_MAX_HEADS,
  * count <= PF_STATIC_MAX_BLOCKS, n_c <= PF_STATIC_MAX_NC; larger sizes
  * return PF_ERR_CAPACITY before any device work.
  * The first call on a device looks up the array's device address with that
- * device current (make that first call before any stream capture).  Every
+ * device current (make that first call before any stream capture); the
+ * address is kept for the process, so a cudaDeviceReset of that device
+ * leaves it stale (do not call this again on a device after resetting it).  Every
  * call clears what must start at zero and then shares the one array: calls
  * that overlap on the GPU (different streams, or different host threads,
  * on one device) race and must not be made.  Three launches on `stream`

@@ -21,7 +21,7 @@ __all__ = [
     "lib", "library_path", "pf_version", "pf_cache_bytes", "pf_cache_create", "pf_cache_destroy",
     "pf_cache_layer_info", "pf_cache_append_block", "pf_cache_load_mid", "pf_select_mid",
     "pf_rope_shift", "pf_attend", "pf_poll_device_error", "pf_selftest_wait_timeout",
-    "pf_select_mid_static", "pf_select_mid_ex", "SelectOpts",
+    "pf_select_mid_static", "pf_select_mid_ex", "SelectOpts", "pf_attend_step", "pf_finish_block",
     "ROUTE_SCORE", "ROUTE_SCORES_ONLY", "ROUTE_GIVEN", "ROUTE_FIFO",
     "PackedKVCache", "config_for",
 ]
@@ -82,9 +82,10 @@ class LayerInfo(ctypes.Structure):
 
 
 def _build_from_sources() -> None:
-    """A checkout without the built library but with its sources: compile it
-    (nvcc, sm_100a) before loading.  build.py is loaded by path so that this
-    package is not imported again; a failed build raises."""
+    """A checkout with the library's sources: compile the library (nvcc,
+    sm_100a) if it is missing or older than a source, before loading.
+    build.py is loaded by path so that this package is not imported again; a
+    failed build raises."""
     from importlib.util import module_from_spec, spec_from_file_location
     spec = spec_from_file_location("_packed_kv_cache_b200_build", os.path.join(_HERE, "build.py"))
     mod = module_from_spec(spec)
@@ -93,7 +94,7 @@ def _build_from_sources() -> None:
 
 
 def _load():
-    if not os.path.exists(library_path) and os.path.isdir(os.path.join(_HERE, "csrc")):
+    if os.path.isdir(os.path.join(_HERE, "csrc")):
         _build_from_sources()
     if not os.path.exists(library_path):
         raise ImportError(f"{library_path} is missing: build it with `python -m packed_kv_cache_b200.build`")
@@ -116,6 +117,9 @@ def _load():
         "pf_poll_device_error": ([vp, vp, ctypes.POINTER(u32)], i32),
         "pf_selftest_wait_timeout": ([vp, u32, vp], i32),
         "pf_select_mid_static": ([vp, i32, i32, i32, vp, i32, i32, i32, i32, i32, vp, vp, vp], i32),
+        "pf_attend_step": ([vp, i32, i32, vp, vp, vp, vp, vp, vp], i32),
+        "pf_finish_block": ([vp, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
+                             ctypes.POINTER(vp), ctypes.POINTER(i32), vp], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -272,6 +276,36 @@ def pf_attend(handle, layer, Q, K_cur, V_cur, O, lse=None, stream=None) -> None:
                                       _dev(O, "O"), _dev(lse, "lse"), _stream(stream)))
 
 
+def pf_attend_step(handle, layer, step, Q, K_cur, V_cur, O, lse=None, stream=None) -> None:
+    """One layer's attention at denoising step `step` of the current block:
+    the selection is made at step 0 and reused by the later steps
+    (PackForcing (arXiv), "Implementation Details"; digest, limitations
+    paragraph)."""
+    _check("pf_attend_step", lib.pf_attend_step(handle, layer, step, _dev(Q, "Q"), _dev(K_cur, "K_cur"),
+                                                _dev(V_cur, "V_cur"), _dev(O, "O"), _dev(lse, "lse"),
+                                                _stream(stream)))
+
+
+def _ptr_array(ts, name):
+    if ts is None:
+        return None
+    arr = (ctypes.c_void_p * len(ts))()
+    for i, t in enumerate(ts):
+        arr[i] = _dev(t, f"{name}[{i}]")
+    return arr
+
+
+def pf_finish_block(handle, K, V, Kc=None, Vc=None, stream=None) -> int:
+    """Append the finished block to every layer (one tensor per layer in each
+    list) and shift every sink by the evicted blocks' frames; returns the
+    blocks evicted per layer."""
+    ev = ctypes.c_int(0)
+    _check("pf_finish_block", lib.pf_finish_block(handle, _ptr_array(K, "K"), _ptr_array(V, "V"),
+                                                  _ptr_array(Kc, "Kc"), _ptr_array(Vc, "Vc"), ctypes.byref(ev),
+                                                  _stream(stream)))
+    return ev.value
+
+
 def pf_poll_device_error(handle, stream=None) -> int:
     """Synchronise `stream` and read (then clear) the cache's device error
     word; raises PF_ERR_TIMEOUT if a bounded wait gave up."""
@@ -289,7 +323,14 @@ def pf_selftest_wait_timeout(handle, timeout_us: int, stream=None) -> None:
 def pf_select_mid_static(Q, batch, n, heads, pool_k, pool_slots, n_c, head, count, n_top, sel_out,
                          scores_out=None, stream=None) -> None:
     """Selection with no device allocation (scratch in a fixed array inside
-    the library): for callers that cannot allocate device memory."""
+    the library): for callers that cannot allocate device memory.  Tensors
+    of the wrong element type, or smaller than the sizes say, are refused
+    before the call (an address given as an int is passed as it is)."""
+    D = 128
+    _expect(Q, "Q", torch.bfloat16, batch * n * heads * D)
+    _expect(pool_k, "pool_k", torch.bfloat16, batch * pool_slots * n_c * heads * D)
+    _expect(sel_out, "sel_out", torch.int32, batch * min(n_top, count))
+    _expect(scores_out, "scores_out", torch.float32, batch * count)
     _check("pf_select_mid_static", lib.pf_select_mid_static(
         _dev(Q, "Q"), batch, n, heads, _dev(pool_k, "pool_k"), pool_slots, n_c, head, count, n_top,
         _dev(sel_out, "sel_out"), _dev(scores_out, "scores_out"), _stream(stream)))
@@ -389,6 +430,32 @@ class PackedKVCache:
             O = torch.empty_like(Q)
         pf_attend(self.handle, layer, Q, K_cur, V_cur, O, lse, stream)
         return O
+
+    def attend_step(self, layer, step, Q, K_cur, V_cur, O=None, lse=None, stream=None) -> torch.Tensor:
+        """Attention at denoising step `step` (selection at step 0, reused
+        after; see pf_attend_step)."""
+        need = self._rows(self._n())
+        for t, name in ((Q, "Q"), (K_cur, "K_cur"), (V_cur, "V_cur"), (O, "O")):
+            _expect(t, name, torch.bfloat16, need)
+        _expect(lse, "lse", torch.float32, need // self.cfg.head_dim)
+        if O is None:
+            O = torch.empty_like(Q)
+        pf_attend_step(self.handle, layer, step, Q, K_cur, V_cur, O, lse, stream)
+        return O
+
+    def finish_block(self, K, V, Kc=None, Vc=None, stream=None) -> int:
+        """Append the final block to every layer and shift the sinks (see
+        pf_finish_block).  K, V, Kc, Vc: one tensor per layer."""
+        L = self.cfg.layers
+        for ts, name, rows in ((K, "K", self._n()), (V, "V", self._n()), (Kc, "Kc", self._n_c()),
+                               (Vc, "Vc", self._n_c())):
+            if ts is None:
+                continue
+            if len(ts) != L:
+                raise ValueError(f"{name} must hold one tensor per layer ({L})")
+            for t in ts:
+                _expect(t, name, torch.bfloat16, self._rows(rows))
+        return pf_finish_block(self.handle, K, V, Kc, Vc, stream)
 
     def poll_device_error(self, stream=None) -> int:
         """See pf_poll_device_error."""

@@ -43,14 +43,10 @@ __global__ void __launch_bounds__(256) copy_runs_kernel(const CopyRuns runs) {
 cudaError_t launch_copy(const CopyRuns& runs, cudaStream_t st) {
   const long long total = runs.start[runs.n];
   if (total <= 0) return cudaSuccess;
-  static int grid_cap = 0;
-  if (grid_cap == 0) {
-    int dev = 0, sms = 148, per_sm = 1;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, copy_runs_kernel, 256, 0);
-    grid_cap = sms * (per_sm > 0 ? per_sm : 1);
-  }
+  static PerDevice cap;
+  int grid_cap = 0;
+  cudaError_t e = cap.get(&grid_cap, [](int dev, int* v) { return one_wave_grid(copy_runs_kernel, dev, v); });
+  if (e != cudaSuccess) return e;
   const long long want = (total + 1023) / 1024;
   const int grid = static_cast<int>(want < grid_cap ? want : grid_cap);
   copy_runs_kernel<<<grid, 256, 0, st>>>(runs);

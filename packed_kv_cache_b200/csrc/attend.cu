@@ -48,10 +48,7 @@ namespace {
 constexpr int kBM = 128;           // query rows per tile
 constexpr int kBN = 128;           // keys per tile
 constexpr int kSub = 32;           // rows per TMA sub-box
-#ifndef PF_ATTEND_K_STAGES
-#define PF_ATTEND_K_STAGES 3
-#endif
-constexpr int kKStages = PF_ATTEND_K_STAGES;  // K ring depth
+constexpr int kKStages = 3;                   // K ring depth
 constexpr int kVStages = 2;                   // V ring depth
 constexpr int kThreads = 384;
 constexpr uint32_t kTileBytes = kBN * kHeadDim * 2;   // 32 KB
@@ -59,36 +56,6 @@ constexpr uint32_t kHalfBytes = kTileBytes / 2;       // 64 dims x 128 rows
 constexpr uint32_t kSubBytes = kSub * 128;            // one sub-box, one 64-dim half
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int kRotThreads = 64;   // warps 2-3
-// Before S_t of the next tile is written over P_t, wait until the P_t V MMA
-// that reads P_t has completed.  Off by default: tcgen05.mma operations
-// issued by one thread execute in issue order.
-#ifndef PF_ATTEND_DRAIN
-#define PF_ATTEND_DRAIN 0
-#endif
-constexpr bool kDrainBeforeOverwrite = PF_ATTEND_DRAIN != 0;
-// The MMA issuer polls both query tiles' P barriers and serves the first
-// ready (1; measured slower: the spinning thread takes issue slots from the
-// softmax warps), or waits for tile 0 then tile 1 (0).
-#ifndef PF_ATTEND_MMA_POLL
-#define PF_ATTEND_MMA_POLL 0
-#endif
-// The two query tiles' exponential phases alternate: tile 1's for K/V tile j
-// starts once tile 0's P_j is ready, tile 0's for tile j+1 once tile 1's P_j
-// is.  Their softmaxes then share the special-function unit in turns and
-// each tile's MMAs run during the other tile's softmax.  Without the gate
-// the two tiles can fall into step (after a run of masked tiles, or from the
-// start): both softmaxes contend for the unit and both tiles' MMAs queue
-// back to back (~1.5x the time per K/V tile).
-#ifndef PF_ATTEND_SLOT_GATE
-#define PF_ATTEND_SLOT_GATE 0
-#endif
-constexpr bool kSlotGate = PF_ATTEND_SLOT_GATE != 0;
-// One exponential pair in kPolyPeriod is evaluated by ex2_poly_x2 (FMA and
-// integer pipes), the others by the special-function unit (0 = never).
-#ifndef PF_ATTEND_POLY_PERIOD
-#define PF_ATTEND_POLY_PERIOD 0
-#endif
-constexpr int kPolyPeriod = PF_ATTEND_POLY_PERIOD;
 
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr uint32_t kOffQ = 0;                                   // 2 tiles
@@ -104,7 +71,6 @@ struct Bars {
   uint64_t k_ready[kKStages];   // K tile rotated (only used when rotate_sink)
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2], o_final[2];
-  uint64_t drain;
   uint32_t tmem_base;
   int abort;
   int merge;
@@ -250,16 +216,11 @@ __device__ __forceinline__ float max64(const uint32_t* x) {
 // stored to 16 TMEM columns at dst; their sum accumulated in rs2.
 __device__ __forceinline__ void exp_chunk(const uint32_t* c, uint32_t dst, uint64_t sl2x2, uint64_t nmbx2,
                                           uint64_t* rs2) {
-  constexpr int period = kPolyPeriod > 0 ? kPolyPeriod : 1;
   uint32_t pk[16];
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
     const uint64_t x = f2_fma((static_cast<uint64_t>(c[2 * e + 1]) << 32) | c[2 * e], sl2x2, nmbx2);
-    uint64_t pp;
-    if (kPolyPeriod > 0 && (e % period) == period - 1)
-      pp = ex2_poly_x2(x);   // FMA pipe: unloads the special-function unit
-    else
-      pp = f2_pack(ex2_approx(f2_lo(x)), ex2_approx(f2_hi(x)));
+    const uint64_t pp = f2_pack(ex2_approx(f2_lo(x)), ex2_approx(f2_hi(x)));
     rs2[e & 1] = f2_add(rs2[e & 1], pp);
     pk[e] = pack_bf16x2(f2_lo(pp), f2_hi(pp));
   }
@@ -313,7 +274,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
       mbar_init(&bars.p_full[t], kBM);
       mbar_init(&bars.o_final[t], 1);
     }
-    mbar_init(&bars.drain, 1);
     bars.abort = 0;
     bars.merge = 0;
     fence_mbar_init();
@@ -416,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
         return mbar_wait_bounded(&k_avail[g % kKStages], (g / kKStages) & 1, abort_flag, p.err,
                                  kDevErrTimeoutBase | site, lim);
       };
-      int kg = 0, vg = 0, drains = 0;
+      int kg = 0, vg = 0;
       bool ok = mbar_wait_bounded(&bars.q_full, 0, abort_flag, p.err, kDevErrTimeoutBase | 4u, lim);
       if (ok) ok = wait_k(kg, 5u);
       if (ok) {
@@ -433,62 +393,21 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
         const int vs = vg % kVStages;
         ok = mbar_wait_bounded(&bars.v_full[vs], (vg / kVStages) & 1, abort_flag, p.err, kDevErrTimeoutBase | 6u,
                                lim);
-#if PF_ATTEND_MMA_POLL
-        // serve the two query tiles in whichever order their P becomes ready
-        {
-          const uint32_t ph = (j - un.j0) & 1;
-          bool served[2] = {false, nq < 2};
-          bool k_ready = !more;
-          const long long t0 = clock64();
-          while (ok && !(served[0] && served[1])) {
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-              if (served[t] || !mbar_test_wait(&bars.p_full[t], ph)) continue;
-              tc_fence_after();
-              issue_pv(t, vs, j == un.j0);
-              if (more) {
-                if (!k_ready) {
-                  ok = wait_k(kg, 10u);
-                  k_ready = ok;
-                  if (!ok) break;
-                  tc_fence_after();
-                }
-                issue_qk(t, kg % kKStages);   // S_t of the next tile overwrites P_t
-                mma_commit(&bars.s_full[t]);
-              }
-              served[t] = true;
-            }
-            if (ok && !(served[0] && served[1])) {
-              if (*abort_flag) ok = false;
-              else if (clock64() - t0 > lim) {
-                *abort_flag = 1;
-                atomicCAS(p.err, 0u, kDevErrTimeoutBase | 7u);
-                ok = false;
-              }
-            }
-          }
-        }
-#else
         for (int t = 0; ok && t < nq; ++t) {
           ok = mbar_wait_bounded(&bars.p_full[t], (j - un.j0) & 1, abort_flag, p.err, kDevErrTimeoutBase | 7u, lim);
           if (!ok) break;
           tc_fence_after();
           issue_pv(t, vs, j == un.j0);
           if (more) {
-            // S_t of the next tile overwrites P_t
-            if (kDrainBeforeOverwrite) {
-              mma_commit(&bars.drain);
-              ok = mbar_wait_bounded(&bars.drain, drains & 1, abort_flag, p.err, kDevErrTimeoutBase | 9u, lim);
-              ++drains;
-            }
-            if (ok && t == 0) ok = wait_k(kg, 10u);
+            // S_t of the next tile overwrites P_t (tcgen05 MMAs issued by
+            // one thread run in issue order: P_t V has read P_t by then)
+            if (t == 0) ok = wait_k(kg, 10u);
             if (!ok) break;
             tc_fence_after();
             issue_qk(t, kg % kKStages);
             mma_commit(&bars.s_full[t]);
           }
         }
-#endif
         if (!ok) break;
         mma_commit(&bars.v_empty[vs]);
         ++vg;
@@ -596,12 +515,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
         l *= alpha;
         rescale_o = j > un.j0;
         m = mt;
-      }
-      if (kSlotGate && nq == 2 && (t == 1 || j > un.j0)) {
-        // take turns with the other query tile (see kSlotGate)
-        const int o = t ^ 1, jj = (t == 1) ? j : j - 1;
-        ok = mbar_wait_bounded(&bars.p_full[o], (jj - un.j0) & 1, abort_flag, p.err, kDevErrTimeoutBase | 15u, lim);
-        if (!ok) break;
       }
       const float mb = (m == -INFINITY) ? 0.f : m;
       const uint64_t sl2x2 = f2_pack(sl2, sl2), nmbx2 = f2_pack(-mb, -mb);
@@ -738,12 +651,13 @@ int attend_tail_chunks(int B, int H, int q_tiles, int n_tiles) {
 }
 
 cudaError_t launch_attend(const AttendParams& p, cudaStream_t st) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  // the kernel's shared-memory limit is raised once per device
+  static PerDevice attr;
+  int unused = 0;
+  cudaError_t e = attr.get(&unused, [](int, int*) {
+    return cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  });
+  if (e != cudaSuccess) return e;
   const long long bh = 1LL * p.B * p.H;
   const long long units = bh * (p.q_tiles / 2) + ((p.q_tiles & 1) ? bh * p.tail_chunks : 0);
   if (units > 0x7fffffffLL) return cudaErrorInvalidValue;

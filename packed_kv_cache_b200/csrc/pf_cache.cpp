@@ -46,8 +46,6 @@ constexpr size_t kAlign = 256;
 constexpr long long kDefaultTimeoutCycles = 4000000000LL;  // about 2 s at 2 GHz
 constexpr int kMaxPoolSlots = 8192;                         // the top-k keeps all scores in shared memory
 
-size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
-
 // attention scratch shared by all layers: split-tail partial outputs, row
 // statistics and tickets
 constexpr size_t kAttendScratchBytes = pf::kAttendPartOBytes + pf::kAttendPartMLBytes + pf::kAttendTicketBytes;
@@ -136,11 +134,14 @@ Geometry geometry(const pf_config* c, bool* overflow) {
   g.recent_bytes = z.bytes(B, c->recent_blocks, g.n, row);
   g.chunk_rows = 32;
   g.chunks_per_block = (g.n_c + g.chunk_rows - 1) / g.chunk_rows;
+  // selection scratch: per-row-chunk query sums, per-slab partial scores of
+  // every slot, and the batch and slab tickets
+  const int slabs = g.HD / pf::kSelSlabCols;
   g.sel_bytes = z.bytes(B, c->n_top > 0 ? c->n_top : 1, 4);
   g.scores_bytes = z.bytes(B, g.slots, 4);
-  g.partial_bytes = z.bytes(B, g.slots, g.chunks_per_block, 4);
-  g.qsum_bytes = z.bytes(B, g.HD, 4);
-  g.ticket_bytes = z.bytes(B, 4, 1);
+  g.partial_bytes = z.bytes(B, g.slots, std::max(g.chunks_per_block, slabs), 4);
+  g.qsum_bytes = z.bytes(B, pf::kSelMaxRowChunks, g.HD, 4);
+  g.ticket_bytes = z.bytes(B, 1 + slabs, 4);
   g.kbar_bytes = z.bytes(B, g.slots, g.HD, 4);
   size_t t = z.mul(2, z.add(z.add(g.sink_bytes, g.pool_bytes), g.recent_bytes));
   t = z.add(t, z.add(z.add(g.sel_bytes, g.scores_bytes), g.partial_bytes));
@@ -161,31 +162,47 @@ struct Layer {
   char *sink_k, *sink_v, *pool_k, *pool_v, *recent_k, *recent_v;
   int32_t* sel;
   float *scores, *partial, *qsum;
-  unsigned* ticket;
+  unsigned* ticket;       // [B] batch tickets, then [B, H * D / 64] slab tickets
   float* kbar;  // [B, slots, H * D] mean key of each pool slot
+  // the attention's tensor maps over this layer's partitions (sink, mid
+  // pool, recent ring), encoded at the layer's first pf_attend: the arena
+  // does not move, so they stay valid for the cache's life
+  bool maps_ready = false;
+  CUtensorMap tm_k[3], tm_v[3];
 };
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+EncodeTiledFn lookup_encode_fn() {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    return reinterpret_cast<EncodeTiledFn>(p);
+  return nullptr;
+}
+
+// looked up once per process (thread-safe initialisation of a local static)
 EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+  static const EncodeTiledFn fn = lookup_encode_fn();
   return fn;
 }
 
 }  // namespace
 
 namespace pf {
+CUresult encode_tiled(CUtensorMap* m, CUtensorMapDataType dtype, int rank, void* base, const cuuint64_t* dims,
+                      const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle swizzle,
+                      CUtensorMapL2promotion l2) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr) return CUDA_ERROR_NOT_SUPPORTED;
+  const cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
+  return fn(m, dtype, static_cast<cuuint32_t>(rank), base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swizzle, l2, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
 int report_error(int status, const char* fmt, ...) {
   char buf[512];
   va_list ap;
@@ -227,17 +244,14 @@ pf_status check_ptr(const void* p, const char* name) {
 // 4-D map (D, H, rows, segs) over a bf16 [segs, rows, H, D] tensor with
 // 64-dim x `box_rows` boxes and 128-byte swizzle.
 pf_status encode_map(CUtensorMap* m, const void* base, int H, long long rows, long long segs, int box_rows) {
-  EncodeTiledFn fn = get_encode_fn();
-  if (fn == nullptr) return fail(PF_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable (driver too old?)");
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(pf::kHeadDim), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(segs)};
   const cuuint64_t rowb = static_cast<cuuint64_t>(pf::kHeadDim) * 2;
   const cuuint64_t strides[3] = {rowb, rowb * H, rowb * H * static_cast<cuuint64_t>(rows)};
   const cuuint32_t box[4] = {64u, 1u, static_cast<cuuint32_t>(box_rows), 1u};
-  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
-  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUresult r = pf::encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                                      box, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+  if (r == CUDA_ERROR_NOT_SUPPORTED) return fail(PF_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable (driver too old?)");
   if (r != CUDA_SUCCESS) return fail(PF_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return PF_OK;
 }
@@ -247,11 +261,14 @@ struct RunBuilder {
   pf::RopeTable tab;
   cudaStream_t st;
   bool f32 = false;  // runs of float32 vectors (cached mean keys) instead of bf16 keys
+  unsigned* dev_err = nullptr;
+  long long timeout_cycles = 0;
   cudaError_t err = cudaSuccess;
   RunBuilder() { runs.n = 0; runs.start[0] = 0; }
   void flush() {
     if (runs.n == 0) return;
-    cudaError_t e = f32 ? pf::launch_rope_shift_f32(runs, tab, st) : pf::launch_rope_shift(runs, tab, st);
+    cudaError_t e = f32 ? pf::launch_rope_shift_f32(runs, tab, st)
+                        : pf::launch_rope_shift(runs, tab, dev_err, timeout_cycles, st);
     if (e != cudaSuccess && err == cudaSuccess) err = e;
     runs.n = 0;
     runs.start[0] = 0;
@@ -598,12 +615,29 @@ pf_status pf_select_mid_ex(pf_cache* c, int layer, const void* Q, const pf_selec
   a.head = Ly.mid_head;
   a.count = Ly.mid_count;
   a.chunk_rows = g.chunk_rows;
-  a.chunks_per_block = 1;   // one partial per block: the dot product with its mean key
+  // one partial score per 64-column slab of the heads used, slab-major
+  const int nslabs = (o.head_hi - o.head_lo) * pf::kHeadDim / pf::kSelSlabCols;
+  a.chunks_per_block = nslabs;
+  a.p_stride = 1;
+  a.k_stride = g.slots;
+  a.partial_ld = nslabs * g.slots;
+  a.slab_ticket = Ly.ticket + cf.batch;
+  {
+    // row chunks per slab: about two CTAs per SM over the whole grid
+    static pf::PerDevice sm_count;
+    int sms = 0;
+    cudaError_t e = sm_count.get(&sms, [](int dev, int* v) {
+      return cudaDeviceGetAttribute(v, cudaDevAttrMultiProcessorCount, dev);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "SM count");
+    const long long per = 1LL * nslabs * cf.batch;
+    long long R = (2LL * sms + per - 1) / per;
+    a.row_chunks = static_cast<int>(std::max(1LL, std::min<long long>(pf::kSelMaxRowChunks, R)));
+  }
   const int rows = (g.n + o.q_stride - 1) / o.q_stride;
   const int heads_norm = o.heads_total > 0 ? o.heads_total : o.head_hi - o.head_lo;
   a.score_scale = static_cast<float>(1.0 / (static_cast<double>(rows) * heads_norm * std::sqrt(128.0)));
   a.partial = Ly.partial;
-  a.partial_ld = g.slots;
   a.scores = Ly.scores;
   a.ticket = Ly.ticket;
   a.n_top = cf.n_top;
@@ -619,11 +653,14 @@ pf_status pf_select_mid_ex(pf_cache* c, int layer, const void* Q, const pf_selec
   switch (o.policy) {
     case PF_ROUTE_SCORE:
     case PF_ROUTE_SCORES_ONLY:
-      e = pf::launch_select(a, st);
+      e = pf::launch_select_cached(a, st);
       break;
     case PF_ROUTE_GIVEN:
       a.partial = const_cast<float*>(o.scores_in);
       a.partial_ld = Ly.mid_count;
+      a.chunks_per_block = 1;
+      a.p_stride = 1;
+      a.k_stride = 1;
       a.score_scale = 1.f;
       e = pf::launch_topk_given(a, st);
       break;
@@ -654,6 +691,8 @@ pf_status pf_rope_shift(pf_cache* c, int layer, unsigned parts, int delta, void*
   const Geometry& g = c->g;
   RunBuilder rb, rm;
   rb.st = static_cast<cudaStream_t>(stream);
+  rb.dev_err = c->err;
+  rb.timeout_cycles = c->timeout_cycles;
   rm.st = rb.st;
   rm.f32 = true;
   rb.tab.pairs = cf.rope_split[0] / 2;
@@ -740,7 +779,7 @@ pf_status pf_attend(pf_cache* c, int layer, const void* Q, const void* K_cur, co
     return s;
   if (O == Q || O == K_cur || O == V_cur) return fail(PF_ERR_ARG, "O must not alias the inputs");
   if (lse != nullptr && reinterpret_cast<uintptr_t>(lse) % 4 != 0) return fail(PF_ERR_ARG, "lse misaligned");
-  const Layer& Ly = c->L[layer];
+  Layer& Ly = c->L[layer];
   const pf_config& cf = c->cfg;
   const Geometry& g = c->g;
   pf::AttendParams p;
@@ -758,22 +797,33 @@ pf_status pf_attend(pf_cache* c, int layer, const void* Q, const void* K_cur, co
   }
   const int B = cf.batch, H = cf.heads;
   const int sink_rows = Ly.sink_filled * g.n;
+  if (!Ly.maps_ready) {
+    // the arena's partitions: encoded once per layer
+    if (cf.sink_blocks > 0) {
+      if ((s = encode_map(&Ly.tm_k[0], Ly.sink_k, H, 1LL * cf.sink_blocks * g.n, B, 32)) != PF_OK) return s;
+      if ((s = encode_map(&Ly.tm_v[0], Ly.sink_v, H, 1LL * cf.sink_blocks * g.n, B, 32)) != PF_OK) return s;
+    }
+    if ((s = encode_map(&Ly.tm_k[1], Ly.pool_k, H, g.n_c, 1LL * B * g.slots, 32)) != PF_OK) return s;
+    if ((s = encode_map(&Ly.tm_v[1], Ly.pool_v, H, g.n_c, 1LL * B * g.slots, 32)) != PF_OK) return s;
+    if ((s = encode_map(&Ly.tm_k[2], Ly.recent_k, H, g.n, 1LL * B * cf.recent_blocks, 32)) != PF_OK) return s;
+    if ((s = encode_map(&Ly.tm_v[2], Ly.recent_v, H, g.n, 1LL * B * cf.recent_blocks, 32)) != PF_OK) return s;
+    Ly.maps_ready = true;
+  }
+  // the caller's tensors: encoded per call
   if ((s = encode_map(&p.tm_q, Q, H, g.n, B, 128)) != PF_OK) return s;
   if ((s = encode_map(&p.tm_k[pf::kPartCur], K_cur, H, g.n, B, 32)) != PF_OK) return s;
   if ((s = encode_map(&p.tm_v[pf::kPartCur], V_cur, H, g.n, B, 32)) != PF_OK) return s;
   if (cf.sink_blocks > 0) {
-    if ((s = encode_map(&p.tm_k[pf::kPartSink], Ly.sink_k, H, 1LL * cf.sink_blocks * g.n, B, 32)) != PF_OK) return s;
-    if ((s = encode_map(&p.tm_v[pf::kPartSink], Ly.sink_v, H, 1LL * cf.sink_blocks * g.n, B, 32)) != PF_OK) return s;
+    p.tm_k[pf::kPartSink] = Ly.tm_k[0];
+    p.tm_v[pf::kPartSink] = Ly.tm_v[0];
   } else {
     p.tm_k[pf::kPartSink] = p.tm_k[pf::kPartCur];
     p.tm_v[pf::kPartSink] = p.tm_v[pf::kPartCur];
   }
-  if ((s = encode_map(&p.tm_k[pf::kPartMid], Ly.pool_k, H, g.n_c, 1LL * B * g.slots, 32)) != PF_OK) return s;
-  if ((s = encode_map(&p.tm_v[pf::kPartMid], Ly.pool_v, H, g.n_c, 1LL * B * g.slots, 32)) != PF_OK) return s;
-  if ((s = encode_map(&p.tm_k[pf::kPartRecent], Ly.recent_k, H, g.n, 1LL * B * cf.recent_blocks, 32)) != PF_OK)
-    return s;
-  if ((s = encode_map(&p.tm_v[pf::kPartRecent], Ly.recent_v, H, g.n, 1LL * B * cf.recent_blocks, 32)) != PF_OK)
-    return s;
+  p.tm_k[pf::kPartMid] = Ly.tm_k[1];
+  p.tm_v[pf::kPartMid] = Ly.tm_v[1];
+  p.tm_k[pf::kPartRecent] = Ly.tm_k[2];
+  p.tm_v[pf::kPartRecent] = Ly.tm_v[2];
   p.O = O;
   p.lse = lse;
   p.B = B;
@@ -821,6 +871,49 @@ pf_status pf_attend(pf_cache* c, int layer, const void* Q, const void* K_cur, co
   if (units > 0x7fffffffLL) return fail(PF_ERR_CAPACITY, "too many work units");
   cudaError_t e = pf::launch_attend(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "attend launch");
+  return PF_OK;
+}
+
+pf_status pf_attend_step(pf_cache* c, int layer, int step, const void* Q, const void* K_cur, const void* V_cur,
+                         void* O, float* lse, void* stream) {
+  pf_status s = check_layer(c, layer);
+  if (s != PF_OK) return s;
+  if (step < 0) return fail(PF_ERR_ARG, "step %d < 0", step);
+  if (step == 0) {
+    // check attention's arguments first, so a refused call selects nothing
+    if ((s = check_ptr(Q, "Q")) != PF_OK || (s = check_ptr(K_cur, "K_cur")) != PF_OK ||
+        (s = check_ptr(V_cur, "V_cur")) != PF_OK || (s = check_ptr(O, "O")) != PF_OK)
+      return s;
+    if (O == Q || O == K_cur || O == V_cur) return fail(PF_ERR_ARG, "O must not alias the inputs");
+    if (lse != nullptr && reinterpret_cast<uintptr_t>(lse) % 4 != 0) return fail(PF_ERR_ARG, "lse misaligned");
+    if ((s = pf_select_mid(c, layer, Q, nullptr, nullptr, stream)) != PF_OK) return s;
+  }
+  return pf_attend(c, layer, Q, K_cur, V_cur, O, lse, stream);
+}
+
+pf_status pf_finish_block(pf_cache* c, const void* const* K, const void* const* V, const void* const* Kc,
+                          const void* const* Vc, int* evicted, void* stream) {
+  if (c == nullptr) return fail(PF_ERR_ARG, "cache is NULL");
+  if (K == nullptr || V == nullptr) return fail(PF_ERR_ARG, "K and V arrays must not be NULL");
+  const pf_config& cf = c->cfg;
+  pf_status s;
+  for (int l = 0; l < cf.layers; ++l) {
+    if ((s = check_ptr(K[l], "K[layer]")) != PF_OK || (s = check_ptr(V[l], "V[layer]")) != PF_OK) return s;
+    const Layer& Ly = c->L[l];
+    if (Ly.sink_filled < cf.sink_blocks || cf.mid_capacity == 0) continue;   // Kc/Vc not needed
+    if (Kc == nullptr || Vc == nullptr) return fail(PF_ERR_ARG, "Kc and Vc arrays must not be NULL");
+    if ((s = check_ptr(Kc[l], "Kc[layer]")) != PF_OK || (s = check_ptr(Vc[l], "Vc[layer]")) != PF_OK) return s;
+  }
+  int ev0 = 0;
+  for (int l = 0; l < cf.layers; ++l) {
+    int ev = 0;
+    s = pf_cache_append_block(c, l, K[l], V[l], Kc ? Kc[l] : nullptr, Vc ? Vc[l] : nullptr, &ev, stream);
+    if (s != PF_OK) return s;
+    if (l == 0) ev0 = ev;
+    else if (ev != ev0) return fail(PF_ERR_STATE, "layer %d evicted %d blocks, layer 0 %d", l, ev, ev0);
+  }
+  if (ev0 > 0 && (s = pf_rope_shift(c, -1, PF_PART_SINK, ev0 * cf.block_frames, stream)) != PF_OK) return s;
+  if (evicted) *evicted = ev0;
   return PF_OK;
 }
 

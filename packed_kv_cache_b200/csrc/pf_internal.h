@@ -6,10 +6,58 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 namespace pf {
 
 constexpr int kHeadDim = 128;
 constexpr int kMaxSegs = 64;
+constexpr int kMaxDevices = 64;
+
+// A launcher's per-device set-up (a kernel attribute raised, a grid size
+// from the device's SM count and the kernel's occupancy), done once per
+// device, with that device current, under a lock.  A process may drive
+// several GPUs from several threads.  The cached results belong to the
+// device's primary context: after cudaDeviceReset they are stale.
+class PerDevice {
+ public:
+  // *out = the value compute(dev, &value) produced for the current device.
+  template <class F>
+  cudaError_t get(int* out, F compute) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu_);
+    if (!done_[dev]) {
+      int v = 0;
+      e = compute(dev, &v);
+      if (e != cudaSuccess) return e;
+      value_[dev] = v;
+      done_[dev] = true;
+    }
+    *out = value_[dev];
+    return cudaSuccess;
+  }
+
+ private:
+  std::mutex mu_;
+  int value_[kMaxDevices] = {};
+  bool done_[kMaxDevices] = {};
+};
+
+// SMs x resident CTAs of `kernel` (256 threads, no dynamic shared memory)
+// on device dev: a grid that fills the GPU in one wave.
+template <class K>
+cudaError_t one_wave_grid(K kernel, int dev, int* out) {
+  int sms = 0, per_sm = 0;
+  cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, 0);
+  if (e != cudaSuccess) return e;
+  *out = sms * (per_sm > 0 ? per_sm : 1);
+  return cudaSuccess;
+}
 
 // Device error codes written to the cache's error word.
 constexpr unsigned kDevErrTimeoutBase = 0x100u;  // | site id
@@ -65,7 +113,10 @@ __device__ __forceinline__ void rope_rotate_word(uint4& w, int word, const RopeT
 }
 #endif
 
-cudaError_t launch_rope_shift(const RowRuns& runs, const RopeTable& tab, cudaStream_t st);
+// bf16 key vectors, in place; a wait that gives up records a timeout in
+// *err (the cache's error word) after timeout_cycles SM clocks.
+cudaError_t launch_rope_shift(const RowRuns& runs, const RopeTable& tab, unsigned* err, long long timeout_cycles,
+                              cudaStream_t st);
 // The same rotation of float32 128-dim vectors (cached mean keys); runs count vectors.
 cudaError_t launch_rope_shift_f32(const RowRuns& runs, const RopeTable& tab, cudaStream_t st);
 
@@ -81,10 +132,18 @@ struct CopyRuns {
 cudaError_t launch_copy(const CopyRuns& runs, cudaStream_t st);
 
 // ------------------------------------------------------------- selection
+// The cache path's selection runs as one kernel over 64-column slabs of the
+// H * D query vector: kSelRowChunks chunks of query rows per slab at most.
+constexpr int kSelSlabCols = 64;
+constexpr int kSelMaxRowChunks = 8;
+
 struct SelectArgs {
   const void* Q;        // [B, n, H, D] bf16
   int B, n, HD;         // HD = H * D
-  float* qsum;          // [B, HD] accumulator, zero on entry, left zero on exit
+  float* qsum;          // [B, HD] query sums (streaming path); [B, kSelMaxRowChunks, HD]
+                        // per-row-chunk partial sums (cache path)
+  unsigned* slab_ticket;  // cache path: [B, HD / kSelSlabCols], zero on entry, left zero on exit
+  int row_chunks;       // cache path: row chunks per slab (1 .. kSelMaxRowChunks)
   const void* pool_k;   // [B, slots, n_c, H, D] bf16
   const float* kbar;    // [B, slots, HD] mean key per pool slot, or null: stream pool_k
   int slots, n_c;
@@ -92,7 +151,9 @@ struct SelectArgs {
   int chunk_rows;       // pool rows per scoring CTA
   int chunks_per_block;
   float score_scale;    // 1 / (n * n_c * H * sqrt(D))
-  float* partial;       // [B, slots, chunks_per_block]
+  float* partial;       // partial scores: element (block age q, part k) of batch item b at
+                        // b * partial_ld + q * p_stride + k * k_stride, k < chunks_per_block
+  int p_stride, k_stride;
   float* scores;        // [B, slots] by age
   unsigned* ticket;     // [B], zero on entry, left zero on exit
   int n_top;
@@ -105,8 +166,11 @@ struct SelectArgs {
   int partial_ld;       // per-batch-item length of `partial`
 };
 
-// qpool + scoring (+ top-k unless a.topk == 0).
+// qpool + scoring of the streamed compressed keys (+ top-k unless a.topk == 0).
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
+// The same from the cached mean keys (a.kbar), as one kernel: query pooling
+// and the partial dot products per slab, then the top-k (unless a.topk == 0).
+cudaError_t launch_select_cached(const SelectArgs& a, cudaStream_t st);
 // Top-k of given scores: a.partial holds [B, partial_ld] scores by age
 // (chunks_per_block = 1, score_scale = 1).
 cudaError_t launch_topk_given(const SelectArgs& a, cudaStream_t st);
@@ -161,6 +225,13 @@ constexpr size_t kAttendTicketBytes = size_t(kAttendMaxTailSlots) * 4;
 int attend_tail_chunks(int B, int H, int q_tiles, int n_tiles);
 
 cudaError_t launch_attend(const AttendParams& p, cudaStream_t st);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (element
+// strides 1, no interleave, out-of-bounds elements read as zero);
+// CUDA_ERROR_NOT_SUPPORTED if the driver does not provide it.
+CUresult encode_tiled(CUtensorMap* m, CUtensorMapDataType dtype, int rank, void* base, const cuuint64_t* dims,
+                      const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle swizzle,
+                      CUtensorMapL2promotion l2);
 
 // Record a failure message for pf_last_error() and return the status.
 int report_error(int status, const char* fmt, ...);

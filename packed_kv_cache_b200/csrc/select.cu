@@ -10,15 +10,19 @@
 //   S[b, p] = qsum[b] . kbar[b, p] / (n H sqrt(D)),  kbar = the block's mean key,
 // so when the cache keeps each compressed block's mean key (computed once,
 // when the block enters the pool) scoring reads 6 KB per block instead of its
-// n_c keys (score_mean_kernel).  Otherwise (the allocation-free entry point)
-// two HBM-streaming kernels:
-//   1. qpool: the columns of Q[b] summed over the block's rows into qsum[b]
-//      (shared by both paths).
+// n_c keys.  That path is one kernel (select_cached_kernel): CTAs own a
+// 64-column slab of the H*D query vector and a chunk of the query rows; each
+// sums its rows' columns, the last row chunk of a slab (ticket) adds the
+// chunks and takes the slab's part of every block's dot product with its
+// mean key, and the last slab of a batch item (ticket) adds the slabs' parts
+// in a fixed order, runs an exact radix select of the n_top largest scores
+// (ties to the older block), writes the selection in ascending age, and
+// clears its tickets.  The allocation-free entry point has no cached means
+// and streams the keys with two kernels:
+//   1. qpool: the columns of Q[b] summed over the block's rows into qsum[b].
 //   2. score: one CTA per 32-row chunk of a pool block, a dot product with
-//      qsum[b]; the last CTA of batch item b (ticket counter) sums the
-//      chunks of each block in a fixed order, runs an exact radix select of
-//      the n_top largest scores (ties to the older block), writes the
-//      selection in ascending age, and clears its ticket.
+//      qsum[b]; the last CTA of batch item b (ticket counter) adds the chunks
+//      of each block in a fixed order and runs the same top-k.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -146,9 +150,9 @@ __device__ void select_tail(const SelectArgs& a, int b, uint32_t* keys) {
   const int t = threadIdx.x;
   const int count = a.count;
   for (int q = t; q < count; q += kThreads) {
-    const float* pp = a.partial + static_cast<long long>(b) * a.partial_ld + static_cast<long long>(q) * a.chunks_per_block;
+    const float* pp = a.partial + static_cast<long long>(b) * a.partial_ld + static_cast<long long>(q) * a.p_stride;
     float s = 0.f;
-    for (int k = 0; k < a.chunks_per_block; ++k) s += __ldcg(pp + k);
+    for (int k = 0; k < a.chunks_per_block; ++k) s += __ldcg(pp + static_cast<long long>(k) * a.k_stride);
     s *= a.score_scale;
     keys[q] = order_key(s);
     a.scores[static_cast<long long>(b) * a.slots + q] = s;
@@ -284,54 +288,115 @@ __global__ void __launch_bounds__(kThreads, 5) score_kernel(const SelectArgs a) 
   select_tail(a, b, keys);
 }
 
-// Factored scoring: S[b, p] = qsum[b] . kbar[b, slot(p)] * scale, one warp per
-// block, kbar the block's mean key (float32, kept with the pool).
-__global__ void __launch_bounds__(kThreads) score_mean_kernel(const SelectArgs a) {
+// The cache path's selection in one kernel.  CTA (x, b): slab x / R of the
+// score's column range [d_lo, d_hi) (kSelSlabCols columns), row chunk x % R
+// of the pooled query rows (R = a.row_chunks).
+//  1. column sums of the chunk's rows over the slab -> qsum[b, chunk, slab];
+//  2. the last chunk of the slab (slab ticket) adds the R chunk sums (in
+//     chunk order) and forms, for every live block, the slab's part of the
+//     dot product with the block's mean key -> partial[b, slab, age];
+//  3. the last slab (batch ticket) adds the parts (in slab order) and runs
+//     the top-k (select_tail).
+constexpr int kSelLoads = 8;   // row loads in flight per thread in step 1
+__global__ void __launch_bounds__(kThreads, 3) select_cached_kernel(const SelectArgs a) {
   extern __shared__ float smem[];
-  float* qs = smem;                                           // [HD] qsum[b]
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + a.HD);  // [count], used by the last CTA
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem);   // [count], the last CTA's top-k
+  __shared__ float red[kThreads / 32][kSelSlabCols];
+  __shared__ float qs[kSelSlabCols];
   __shared__ unsigned is_last;
   const int b = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int p = blockIdx.x * (kThreads / 32) + warp;
-  for (int i = threadIdx.x; i < a.HD; i += kThreads) qs[i] = a.qsum[static_cast<long long>(b) * a.HD + i];
-  __syncthreads();
-  if (p < a.count) {
-    const int slot = (a.head + p) % a.slots;
-    const float4* q = reinterpret_cast<const float4*>(qs);
-    // elements [d_lo, d_hi) of the mean key: the heads that enter the score
-    const float4* k = reinterpret_cast<const float4*>(a.kbar + (static_cast<long long>(b) * a.slots + slot) * a.HD);
-    const int nv = a.d_hi / 4;
-    float acc = 0.f;
-    // eight 16-byte loads of the mean key in flight per lane
-    for (int i0 = a.d_lo / 4 + lane; i0 < nv; i0 += 32 * 8) {
-      float4 y[8];
+  const int R = a.row_chunks;
+  const int slab = blockIdx.x / R, rc = blockIdx.x - slab * R;
+  const int nslabs = gridDim.x / R;
+  const int col0 = a.d_lo + slab * kSelSlabCols;
+  const int G = a.HD / 8;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  // ---- 1. column sums: thread t owns 16-byte group t % 8 of the slab in row phase t / 8
+  {
+    const int g = t & 7, phase = t >> 3;
+    constexpr int kPhases = kThreads / 8;
+    const int nr = (a.n + a.q_stride - 1) / a.q_stride;   // pooled rows 0, q_stride, 2 q_stride, ...
+    const int r_lo = static_cast<int>(static_cast<long long>(rc) * nr / R);
+    const int r_hi = static_cast<int>(static_cast<long long>(rc + 1) * nr / R);
+    const uint4* Q = static_cast<const uint4*>(a.Q) + static_cast<long long>(b) * a.n * G + col0 / 8 + g;
+    const long long row_step = static_cast<long long>(a.q_stride) * G;
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int r = r_lo + phase; r < r_hi; r += kSelLoads * kPhases) {
+      uint4 w[kSelLoads];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + 32 * u;
-        y[u] = i < nv ? __ldg(k + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int k = 0; k < kSelLoads; ++k) {
+        const int rr = r + k * kPhases;
+        w[k] = rr < r_hi ? __ldg(Q + rr * row_step) : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + 32 * u;
-        if (i < nv) {
-          const float4 x = q[i];
-          acc = fmaf(x.x, y[u].x, fmaf(x.y, y[u].y, fmaf(x.z, y[u].z, fmaf(x.w, y[u].w, acc))));
-        }
-      }
+      for (int k = 0; k < kSelLoads; ++k) acc_bf16x8(acc, w[k]);
     }
+    // the four row phases of a warp hold the same group: lanes g, g + 8, g + 16, g + 24
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) a.partial[static_cast<long long>(b) * a.partial_ld + p] = acc;
+    for (int e = 0; e < 8; ++e) {
+      acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 8);
+      acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+    }
+    if (lane < 8) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) red[warp][lane * 8 + e] = acc[e];
+    }
+    __syncthreads();
+    if (t < kSelSlabCols) {
+      float sum = 0.f;
+#pragma unroll
+      for (int w = 0; w < kThreads / 32; ++w) sum += red[w][t];
+      a.qsum[(static_cast<long long>(b) * kSelMaxRowChunks + rc) * a.HD + col0 + t] = sum;
+      __threadfence();
+    }
+    __syncthreads();
+    if (t == 0) {
+      __threadfence();
+      unsigned* tk = a.slab_ticket + static_cast<long long>(b) * (a.HD / kSelSlabCols) + slab;
+      is_last = (atomicAdd(tk, 1u) == static_cast<unsigned>(R - 1)) ? 1u : 0u;
+      if (is_last) *tk = 0u;   // every chunk of this slab has arrived: ready for the next launch
+    }
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+  }
+  // ---- 2. this slab's part of every live block's score
+  if (t < kSelSlabCols) {
+    float sum = 0.f;
+    for (int c = 0; c < R; ++c) sum += __ldcg(a.qsum + (static_cast<long long>(b) * kSelMaxRowChunks + c) * a.HD + col0 + t);
+    qs[t] = sum;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
+  {
+    const float4* q4 = reinterpret_cast<const float4*>(qs);
+    float* part = a.partial + static_cast<long long>(b) * a.partial_ld + static_cast<long long>(slab) * a.k_stride;
+    // one block per thread per step: its 256 bytes (16 loads) in flight
+    for (int p = t; p < a.count; p += kThreads) {
+      int slot = a.head + p;
+      if (slot >= a.slots) slot -= a.slots;
+      const float4* k4 = reinterpret_cast<const float4*>(a.kbar + (static_cast<long long>(b) * a.slots + slot) * a.HD + col0);
+      float4 y[kSelSlabCols / 4];
+#pragma unroll
+      for (int i = 0; i < kSelSlabCols / 4; ++i) y[i] = __ldg(k4 + i);
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < kSelSlabCols / 4; ++i) {
+        const float4 x = q4[i];
+        acc = fmaf(x.x, y[i].x, fmaf(x.y, y[i].y, fmaf(x.z, y[i].z, fmaf(x.w, y[i].w, acc))));
+      }
+      part[p] = acc;
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (t == 0) {
     __threadfence();
-    is_last = (atomicAdd(&a.ticket[b], 1u) == gridDim.x - 1u) ? 1u : 0u;
+    is_last = (atomicAdd(&a.ticket[b], 1u) == static_cast<unsigned>(nslabs - 1)) ? 1u : 0u;
   }
   __syncthreads();
   if (!is_last) return;
   __threadfence();
+  // ---- 3. scores (slab parts added in slab order) and the top-k
   select_tail(a, b, keys);
 }
 
@@ -394,17 +459,6 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
   qpool_kernel<<<g1, kQcThreads, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (a.kbar != nullptr) {
-    // factored: one warp per block against its cached mean key
-    const size_t smem = static_cast<size_t>(a.HD) * 4 + static_cast<size_t>(a.count) * 4;
-    if (smem > 48 * 1024) {
-      e = cudaFuncSetAttribute(score_mean_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-    }
-    dim3 g2((a.count + kThreads / 32 - 1) / (kThreads / 32), a.B);
-    score_mean_kernel<<<g2, kThreads, smem, st>>>(a);
-    return cudaGetLastError();
-  }
   const size_t smem = static_cast<size_t>(a.HD) * 4 + static_cast<size_t>(a.count) * 4;
   if (smem > 48 * 1024) {
     e = cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -412,6 +466,21 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
   }
   dim3 g2(a.count * a.chunks_per_block, a.B);
   score_kernel<<<g2, kThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_cached(const SelectArgs& a, cudaStream_t st) {
+  if (a.count <= 0) return cudaSuccess;
+  const int nslabs = (a.d_hi - a.d_lo) / kSelSlabCols;
+  if (nslabs <= 0 || a.row_chunks < 1 || a.row_chunks > kSelMaxRowChunks || a.chunks_per_block != nslabs)
+    return cudaErrorInvalidValue;
+  const size_t smem = static_cast<size_t>(a.count) * 4;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(select_cached_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  select_cached_kernel<<<dim3(nslabs * a.row_chunks, a.B), kThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -518,7 +587,7 @@ extern "C" pf_status pf_select_mid_static(const void* Q, int batch, int n, int h
   if (static_cast<long long>(batch) * pool_slots > kStaticBlocks * static_cast<long long>(kStaticBatch))
     return static_cast<pf_status>(report_error(PF_ERR_CAPACITY, "batch * pool_slots must be <= %d",
                                                kStaticBlocks * kStaticBatch));
-  if (count == 0 || n_top == 0) return PF_OK;
+  if (count == 0 || (n_top == 0 && scores_out == nullptr)) return PF_OK;
   StaticSelectScratch* sc = nullptr;
   cudaError_t e = static_scratch(&sc);
   if (e != cudaSuccess)
@@ -555,8 +624,12 @@ extern "C" pf_status pf_select_mid_static(const void* Q, int batch, int n, int h
   a.q_stride = 1;
   a.d_lo = 0;
   a.d_hi = HD;
-  a.topk = 1;
+  a.topk = n_top > 0 ? 1 : 0;   // n_top == 0: the scores only
   a.partial_ld = pool_slots * a.chunks_per_block;
+  a.p_stride = a.chunks_per_block;
+  a.k_stride = 1;
+  a.slab_ticket = nullptr;
+  a.row_chunks = 1;
   e = launch_select(a, st);
   if (e != cudaSuccess)
     return static_cast<pf_status>(report_error(PF_ERR_CUDA, "select launch: %s", cudaGetErrorString(e)));
