@@ -60,9 +60,12 @@ def test_cache_bytes_layout(pf):
     al = lambda x: (x + 255) // 256 * 256  # noqa: E731
     slots = wl.mid_capacity + wl.recent_blocks
     cpb = (182 + 31) // 32
+    slabs = 12 * 128 // 64                  # the selection's 64-column slabs of the H * D vector
     per_layer = (2 * (al(2 * 6240 * row) + al(slots * 182 * row) + al(6240 * row))
-                 + al(16 * 4) + al(slots * 4) + al(slots * cpb * 4) + al(12 * 128 * 4) + al(4)
-                 + al(slots * 1536 * 4))   # mean key of every pool slot
+                 + al(16 * 4) + al(slots * 4) + al(slots * max(cpb, slabs) * 4)
+                 + al(8 * 12 * 128 * 4)     # query sums of up to 8 row chunks
+                 + al((1 + slabs) * 4)      # batch and slab tickets
+                 + al(slots * 1536 * 4))    # mean key of every pool slot
     # shared attention scratch: 256 split-tail slots of 128x128 fp32 partial
     # outputs, their row max / row sum, and 256 tickets
     scratch = 256 * 128 * 128 * 4 + 256 * 2 * 128 * 4 + 256 * 4
@@ -246,6 +249,19 @@ def test_cache_methods_refuse_wrong_dtypes_and_short_buffers(pf):
     refused(lambda: cache.append_block(0, Q[:, :-1], Q), "K has")
     refused(lambda: cache.append_block(0, Q, Q, bf(B, nc - 1, H, D), bf(B, nc, H, D)), "Kc has")
     refused(lambda: cache.load_mid(0, bf(B, 3, nc, H, D), bf(B, 2, nc, H, D)), "Vc has")
+    # the allocation-free selection: sizes come from its arguments
+    P, slots = 13, 16
+    pool = bf(B, slots, nc, H, D)
+    sel = torch.zeros((B, 5), dtype=torch.int32)
+    static = lambda **kw: pf.pf_select_mid_static(  # noqa: E731
+        kw.get("Q", Q), B, n, H, kw.get("pool", pool), slots, nc, 3, P, 5, kw.get("sel", sel), kw.get("sc"))
+    refused(lambda: static(Q=Q[:, :-1]), "Q has")
+    refused(lambda: static(Q=Q.float()), "Q must be torch.bfloat16")
+    refused(lambda: static(pool=pool[:, :-1]), "pool_k has")
+    refused(lambda: static(sel=sel[:, :-1]), "sel_out has")
+    refused(lambda: static(sel=sel.long()), "sel_out must be")
+    refused(lambda: static(sc=torch.zeros((B, P - 1))), "scores_out has")
+    refused(lambda: static(sc=torch.zeros((B, P))), "CUDA tensor")
 
 
 def _hold_build_lock(q):

@@ -172,6 +172,46 @@ def test_selection_after_rotating_the_pool(pf, name):
             assert np.array_equal(sel.cpu().numpy()[b], sel_ref[b])
 
 
+@pytest.mark.parametrize("name", ["ragged_b", "layer"])
+def test_cached_mean_keys_after_many_mid_shifts(pf, name):
+    # A shift rounds the pool's stored keys to bf16 and rotates each block's
+    # cached float32 mean key without rounding.  After 24 shifts the cached
+    # means are the means of the keys rotated exactly by the total shift
+    # (the method's k' = k e^{i theta delta}), so the selection's scores must
+    # match the oracle's scores of those keys tightly; the stored keys have
+    # drifted from them by 24 bf16 roundings, which is bounded here too.
+    wl = _wl(name)
+    d = synth.make_layer(wl, seed_for(name))
+    cache = build_cache(pf, wl, d)
+    rng = np.random.default_rng(11)
+    total = 0
+    for _ in range(24):
+        delta = int(rng.integers(1, 65))
+        cache.rope_shift(0, pf.PART_MID, delta)
+        total += delta
+    B, P, nc, H, D = wl.batch, wl.pool_blocks, wl.n_c, wl.heads, wl.head_dim
+    info = cache.info(0)
+    k = min(wl.n_top, P)
+    sel = torch.full((B, k), -1, dtype=torch.int32, device="cuda")
+    sc = torch.zeros((B, P), dtype=torch.float32, device="cuda")
+    cache.select_mid(0, d["Q"].cuda(), sel, sc)
+    torch.cuda.synchronize()
+    S_exact = oracle.select_scores(d["Q"], oracle.rope_shift(d["mid_K"], total))
+    scale = np.abs(S_exact).max(axis=1, keepdims=True)
+    assert np.max(np.abs(sc.cpu().numpy() - S_exact) / scale) < 2e-5
+    margin = oracle.selection_margin(S_exact, wl.n_top)
+    sel_ref = oracle.select_topk(S_exact, wl.n_top)
+    for b in range(B):
+        if margin[b] >= 1e-3:
+            assert np.array_equal(sel.cpu().numpy()[b], sel_ref[b])
+    # the keys as stored: within the accumulated rounding of 24 bf16 stores
+    slots, head = info["pool_slots"], info["mid_head"]
+    pool = arena_view(cache, info["pool_k"], (B, slots, nc, H, D)).cpu()
+    live = torch.stack([pool[:, (head + p) % slots] for p in range(P)], 1)
+    S_stored = oracle.select_scores(d["Q"], live)
+    assert np.max(np.abs(S_stored - S_exact) / scale) < 5e-3
+
+
 def test_largest_pool_selection_and_attention(pf):
     # the largest pool a cache allows (8,192 slots = 8,191 live blocks + the
     # recent block's pending copy): the top-k keeps every score in shared memory
@@ -564,6 +604,105 @@ def test_generation_loop_against_oracle_model(pf, fused):
     assert cache.info(0)["total_shift"] == cache.info(0)["evicted"] * Bf
 
 
+def test_block_steps_across_layers_against_oracle_model(pf):
+    """CFG batch 2 (cond + uncond), 2 layers, 4 denoising steps per block,
+    6 blocks.  pf_attend_step selects from the first step's queries and
+    reuses that selection at steps 2-4 while the queries and the current
+    block's K/V change from step to step; pf_finish_block appends the final
+    block to every layer and shifts every sink on eviction.  The oracle keeps
+    its own copy of every layer's partitions; every step's output of every
+    layer is compared with it."""
+    L, S = 2, 4
+    wl = _wl("ragged_a").replace(mid_capacity=3, n_top=2, planted=0, layers=L)
+    B, n, nc, H, D, Bf = wl.batch, wl.n, wl.n_c, wl.heads, wl.head_dim, wl.block_frames
+    cache = pf.PackedKVCache(pf.config_for(wl))
+    model = [{"sinkK": [], "sinkV": [], "mid": [], "recent": []} for _ in range(L)]
+    total_ev = 0
+    for i in range(6):
+        final = [synth.make_block(wl, 7100 + 10 * i + l) for l in range(L)]
+        for step in range(S):
+            for l in range(L):
+                m = model[l]
+                seed = 9100 + 100 * i + 10 * step + l
+                Q = synth.bf16_normal((B, n, H, D), seed)
+                if step == S - 1:
+                    Kcur, Vcur = final[l]["K"], final[l]["V"]
+                else:
+                    Kcur = synth.bf16_normal((B, n, H, D), seed + 50000)
+                    Vcur = synth.bf16_normal((B, n, H, D), seed + 60000)
+                O = cache.attend_step(l, step, Q.cuda(), Kcur.cuda(), Vcur.cuda()).cpu()
+                info = cache.info(l)
+                parts = [(torch.from_numpy(k), v) for k, v in zip(m["sinkK"], m["sinkV"])]
+                if m["mid"]:
+                    if len(m["mid"]) > wl.n_top:
+                        assert info["selection_valid"] == 1
+                        slots = arena_view(cache, info["selection"], (B, wl.n_top), torch.int32).cpu().numpy()
+                        chosen = np.sort((slots - info["mid_head"]) % info["pool_slots"], axis=1)
+                        if step == 0:
+                            q0 = Q
+                            mK = torch.stack([torch.stack([mm[0][b] for mm in m["mid"]]) for b in range(B)])
+                            S_ref = oracle.select_scores(q0, mK)
+                            m["sel_ref"] = (oracle.select_topk(S_ref, wl.n_top), oracle.selection_margin(S_ref, wl.n_top))
+                        sel_ref, margin = m["sel_ref"]
+                        for b in range(B):
+                            if margin[b] >= 1e-3:
+                                assert np.array_equal(chosen[b], sel_ref[b]), (i, step, l, b)
+                    else:
+                        chosen = np.array([list(range(len(m["mid"])))] * B)
+                    for j in range(chosen.shape[1]):
+                        parts.append((torch.stack([m["mid"][chosen[b][j]][0][b] for b in range(B)]),
+                                      torch.stack([m["mid"][chosen[b][j]][1][b] for b in range(B)])))
+                parts += [(r[0], r[1]) for r in m["recent"]]
+                parts.append((Kcur, Vcur))
+                O_ref, _ = oracle.attend(Q, parts)
+                assert_attention_close(O, O_ref, f"block {i} step {step} layer {l}")
+        ev = cache.finish_block([f["K"].cuda() for f in final], [f["V"].cuda() for f in final],
+                                [f["Kc"].cuda() for f in final], [f["Vc"].cuda() for f in final])
+        for l in range(L):
+            m, f = model[l], final[l]
+            if len(m["sinkK"]) < wl.sink_blocks:
+                m["sinkK"].append(oracle.to_f64(f["K"]))
+                m["sinkV"].append(f["V"])
+            else:
+                m["recent"].append((f["K"], f["V"], f["Kc"], f["Vc"]))
+                if len(m["recent"]) > wl.recent_blocks:
+                    old = m["recent"].pop(0)
+                    m["mid"].append((old[2], old[3]))
+                    if len(m["mid"]) > wl.mid_capacity:
+                        m["mid"].pop(0)
+                        assert ev == 1
+            if ev:
+                m["sinkK"] = [oracle.round_bf16(oracle.rope_shift(k, ev * Bf)) for k in m["sinkK"]]
+        total_ev += ev
+    assert total_ev >= 2
+    for l in range(L):
+        assert cache.info(l)["total_shift"] == total_ev * Bf
+
+
+def test_block_step_calls_refuse_bad_arguments(pf):
+    wl = _wl("ragged_a").replace(layers=2)
+    B, n, H, D = wl.batch, wl.n, wl.heads, wl.head_dim
+    cache = pf.PackedKVCache(pf.config_for(wl))
+    blk = synth.make_block(wl, 3)
+    Q = synth.bf16_normal((B, n, H, D), 4).cuda()
+    K, V = blk["K"].cuda(), blk["V"].cuda()
+    with pytest.raises(pf.PFError) as e:
+        cache.attend_step(0, -1, Q, K, V)
+    assert e.value.status_name == "PF_ERR_ARG"
+    with pytest.raises(ValueError):
+        cache.finish_block([K], [V])                      # one tensor per layer
+    with pytest.raises(pf.PFError) as e:                  # a NULL pointer in the array
+        pf.pf_finish_block(cache.handle, [K, 0], [V, V])
+    assert e.value.status_name == "PF_ERR_ARG"
+    assert cache.info(0)["blocks_seen"] == 0 and cache.info(1)["blocks_seen"] == 0   # nothing appended
+    for _ in range(wl.sink_blocks):
+        assert cache.finish_block([K, K], [V, V]) == 0    # sink blocks need no compressed copy
+    with pytest.raises(pf.PFError) as e:                  # now the compressed copies are needed
+        cache.finish_block([K, K], [V, V])
+    assert e.value.status_name == "PF_ERR_ARG"
+    assert cache.info(1)["blocks_seen"] == wl.sink_blocks
+
+
 @pytest.mark.parametrize("name", ["ragged_a", "ragged_c", "layer"])
 def test_sink_rope_in_attention_matches_oracle(pf, name):
     # the sink's shift recorded by pf_rope_shift and applied by pf_attend to
@@ -606,6 +745,27 @@ def test_sink_rope_in_attention_needs_a_full_sink(pf):
     cache.append_block(0, blk["K"].cuda(), blk["V"].cuda())
     cache.rope_shift(0, pf.PART_SINK, 4)
     assert cache.info(0)["total_shift"] == 4
+
+
+# ------------------------------------------------------------------ several devices
+
+def test_two_devices_in_one_process(pf):
+    # each launcher's one-time set-up is per device: a second GPU in the same
+    # process runs the whole path too (a head-sharded layer drives one GPU per
+    # rank, but a single process may also hold caches on several GPUs)
+    if torch.cuda.device_count() < 2:
+        pytest.skip("needs two GPUs")
+    wl, d = _layer("ragged_c")
+    for dev in (0, 1):
+        with torch.cuda.device(dev):
+            cache = build_cache(pf, wl, d, device=f"cuda:{dev}")
+            Q = d["Q"].to(f"cuda:{dev}")
+            s = torch.zeros((wl.batch, wl.n_top), dtype=torch.int32, device=f"cuda:{dev}")
+            cache.select_mid(0, Q, s, None)
+            O = cache.attend(0, Q, d["K_cur"].to(f"cuda:{dev}"), d["V_cur"].to(f"cuda:{dev}"))
+            assert cache.poll_device_error() == 0
+            O_ref, _ = oracle.attend(d["Q"], oracle_context(wl, d, s.cpu().numpy()))
+            assert_attention_close(O.cpu(), O_ref, f"device {dev}")
 
 
 # ------------------------------------------------------------------ failure detection

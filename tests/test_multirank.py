@@ -85,3 +85,73 @@ def test_head_sharded_selection_exchange_on_two_gloo_ranks():
     assert np.array_equal(summed0, summed1) and np.array_equal(sel0, sel1)
     assert np.max(np.abs(summed0 - full)) < 1e-12 * max(1.0, np.max(np.abs(full)))
     assert np.array_equal(sel0, oracle.select_topk(full, 2))
+
+
+class _OracleShardCache:
+    """Stands in for a cache that holds heads [lo, hi) of a layer: its
+    scores-only selection is the oracle's partial score over those heads, and
+    its given-score routing records the oracle's top-k of the scores it gets."""
+
+    def __init__(self, Q, pool_K, lo, hi, n_top):
+        self.Q, self.pool_K, self.lo, self.hi, self.n_top = Q, pool_K, lo, hi, n_top
+        self.routed = None
+
+    def select_mid_ex(self, layer, Q, policy, heads_total=0, scores_in=None, scores_out=None):
+        import oracle
+        if policy == 1:                                   # scores only, this rank's heads
+            part = oracle.select_scores(self.Q[..., self.lo:self.hi, :], self.pool_K[..., self.lo:self.hi, :],
+                                        heads_norm=heads_total)
+            scores_out.copy_(torch.from_numpy(part))
+        elif policy == 2:                                 # top-k of the given scores
+            self.routed = oracle.select_topk(scores_in.numpy(), self.n_top)
+        else:
+            raise AssertionError(policy)
+
+
+def _bench_shard_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import bench
+    import synth
+    bench.dist_init("gloo")
+    wl = synth.WORKLOADS["ragged_c"]                      # 3 heads over the ranks: 2 + 1
+    d = synth.make_layer(wl.replace(pool_blocks=6, planted=2), 21)   # the same layer on every rank
+    H = d["Q"].shape[2]
+    lo, hi = bench.head_shard(H, world, rank)
+    cache = _OracleShardCache(d["Q"], d["mid_K"], lo, hi, 2)
+    scores = torch.zeros((wl.batch, 6), dtype=torch.float64)
+    bench.select_head_sharded(cache, 0, d["Q"], scores, H, lambda t: dist.all_reduce(t, op=dist.ReduceOp.SUM),
+                              1, 2)
+    out[rank] = ((lo, hi), scores.numpy().tolist(), cache.routed.tolist())
+    dist.destroy_process_group()
+
+
+def test_bench_head_sharded_selection_on_two_gloo_ranks():
+    # the bench's own sharded-selection step (scores-only on this rank's heads,
+    # the sum across ranks, the top-k of the sum) against the unsharded oracle
+    world = 2
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.spawn(_bench_shard_worker, args=(world, port, out), nprocs=world, join=True)
+    import numpy as np
+
+    import oracle
+    import synth
+    d = synth.make_layer(synth.WORKLOADS["ragged_c"].replace(pool_blocks=6, planted=2), 21)
+    full = oracle.select_scores(d["Q"], d["mid_K"])
+    assert out[0][0] == (0, 2) and out[1][0] == (2, 3)
+    for r in range(world):
+        assert np.max(np.abs(np.array(out[r][1]) - full)) < 1e-12 * max(1.0, np.max(np.abs(full)))
+        assert np.array_equal(np.array(out[r][2]), oracle.select_topk(full, 2))
+
+
+def test_head_shard_ranges_cover_every_head_once():
+    import bench
+    for H in (1, 3, 12, 16):
+        for world in range(1, H + 1):
+            r = [bench.head_shard(H, world, k) for k in range(world)]
+            assert r[0][0] == 0 and r[-1][1] == H
+            assert all(a[1] == b[0] for a, b in zip(r, r[1:]))
+            sizes = [hi - lo for lo, hi in r]
+            assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1

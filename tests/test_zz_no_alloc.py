@@ -2,12 +2,14 @@
 device memory (a serving process with a fixed device-memory budget and no
 allocation on the request path, or a framework that owns the allocator and
 gives this library no arena).  Its scratch is a fixed array inside the
-library; this checks it against pf_select_mid, through the C ABI, on two
-calls in a row.  The file name makes pytest collect it last."""
+library; this checks it against pf_select_mid and against the oracle,
+through the C ABI, on two calls in a row.  The file name makes pytest
+collect it last."""
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 from _harness import build_cache, seed_for
 
@@ -47,6 +49,39 @@ def test_static_selection_matches_cache_selection(pf, name):
         assert torch.equal(sel, sel_ref)
         assert float(((sc - sc_ref).abs() / scale).max()) < 1e-4
     assert np.array_equal(sel.cpu().numpy(), d["planted"].numpy())
+
+
+@pytest.mark.parametrize("name,slots,head", [("ragged_a", 20, 14), ("layer", 50, 31)])
+def test_static_selection_wrapped_ring_matches_oracle(pf, name, slots, head):
+    # the live blocks run from slot `head` past the end of the ring and on
+    # from slot 0; the other slots hold unrelated keys that must not count
+    wl = synth.WORKLOADS[name]
+    d = synth.make_layer(wl, seed_for(name))
+    B, P, nc, H, D = wl.batch, wl.pool_blocks, wl.n_c, wl.heads, wl.head_dim
+    assert head + P > slots                                   # wraps
+    pool = synth.bf16_normal((B, slots, nc, H, D), 4242)
+    for p in range(P):
+        pool[:, (head + p) % slots] = d["mid_K"][:, p]
+    S_ref = oracle.select_scores(d["Q"], d["mid_K"])
+    sel_ref = oracle.select_topk(S_ref, wl.n_top)
+    assert np.all(oracle.selection_margin(S_ref, wl.n_top) >= 1e-3)
+    Q, pool_d = d["Q"].cuda(), pool.cuda()
+    k = min(wl.n_top, P)
+    scale = np.abs(S_ref).max(axis=1, keepdims=True)
+    for _ in range(2):                       # the second call reuses the array the first one left
+        sel = torch.full((B, k), -1, dtype=torch.int32, device="cuda")
+        sc = torch.zeros((B, P), dtype=torch.float32, device="cuda")
+        pf.pf_select_mid_static(Q, B, wl.n, H, pool_d, slots, nc, head, P, wl.n_top, sel, sc)
+        torch.cuda.synchronize()
+        assert np.array_equal(sel.cpu().numpy(), sel_ref)
+        assert float((np.abs(sc.cpu().numpy() - S_ref) / scale).max()) < 1e-4
+    # n_top = 0: no selection, but the scores are still written
+    sel = torch.full((B, k), -1, dtype=torch.int32, device="cuda")
+    sc = torch.zeros((B, P), dtype=torch.float32, device="cuda")
+    pf.pf_select_mid_static(Q, B, wl.n, H, pool_d, slots, nc, head, P, 0, sel, sc)
+    torch.cuda.synchronize()
+    assert bool((sel == -1).all())
+    assert float((np.abs(sc.cpu().numpy() - S_ref) / scale).max()) < 1e-4
 
 
 def test_static_selection_rejects_sizes_beyond_its_array(pf):
