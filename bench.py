@@ -14,11 +14,23 @@ The metric is packed-cache attention TFLOP/s (attention FLOPs of the step /
 step time) and the per-layer step latency; the roofline line is the
 attention kernel's own time.
 
+The same JSON line carries, under "configs", the other workloads of the
+path, each timed with CUDA events (L2 flushed between iterations) and with
+its own roofline: the 30-layer block of 4 denoising steps at CFG batch 2
+(selection at the first step, reused by the others; append and sink shift
+of every layer after the block), the dense 748,800-key layer, and the
+batch-2 stress layers with a 1,000-block pool (scoring, top-k and the RoPE
+shift of every cached key: the HBM-bound kernels; attention with 16 and 64
+routed blocks; and the streaming scorer of the allocation-free selection,
+which reads the whole compressed pool).
+
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                  [--configs all|none|c2,c3,c4]
 
 For N > 1 run under torchrun: every rank runs an independent replica (its
 own cache and stream of blocks, no data-path collective), time = max over
-ranks, value = the ranks' total work / that time.
+ranks, value = the ranks' total work / that time.  The extra configs run on
+rank 0 only, after the timed region.
 """
 from __future__ import annotations
 
@@ -81,6 +93,27 @@ def rank_seed(base: int, rank: int) -> int:
     return base + 7919 * rank
 
 
+# ---------------------------------------------------------------- head sharding
+
+def head_shard(H: int, world: int, rank: int):
+    """Heads [lo, hi) of this rank: contiguous ranges whose sizes differ by at
+    most one (the first H mod world ranks take one more)."""
+    base, extra = divmod(H, world)
+    lo = rank * base + min(rank, extra)
+    return lo, lo + base + (1 if rank < extra else 0)
+
+
+def select_head_sharded(cache, layer, Q, scores, heads_total, reduce_sum, route_scores_only, route_given):
+    """The selection of a layer whose heads are spread over ranks (one
+    exchange): this rank scores the live blocks on its own heads, divided by
+    the total head count (a partial of the all-head score), the partials are
+    summed across ranks (reduce_sum, in place), and every rank takes the same
+    top-k of the sum with the method's ranking rule."""
+    cache.select_mid_ex(layer, Q, policy=route_scores_only, heads_total=heads_total, scores_out=scores)
+    reduce_sum(scores)
+    cache.select_mid_ex(layer, None, policy=route_given, scores_in=scores)
+
+
 # ---------------------------------------------------------------- helpers
 
 def load_peaks():
@@ -98,47 +131,105 @@ def attention_flops(B, H, Lq, Lk, D=128) -> float:
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+    """SM clock and clock-event reasons of this process's GPU, sampled every
+    ~2 ms by NVML in a host thread (so that even a 20 ms timed region holds
+    several samples), or by ``nvidia-smi -lms 100`` if NVML is unavailable.
+    The GPU is found by its UUID: NVML numbers every GPU of the machine,
+    CUDA only the visible ones."""
 
+    INTERVAL_S = 0.002
     FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, device_index: int):
+        self.device_index = device_index
+        self.rows = []          # (host time, sm MHz, max sm MHz, [reason names])
+        self.thread = None
+        self.stop_flag = False
         self.proc = None
         self.path = None
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(self.device_index).uuid)
+        return pynvml, pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
 
     def start(self):
         try:
+            nv, h = self._nvml_handle()
+        except Exception:
+            nv = None
+        if nv is not None:
+            import threading
+            self.source = "nvml"
+
+            def loop():
+                mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                while not self.stop_flag:
+                    try:
+                        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                        bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.rows.append((time.time(), float(sm), float(mx), reason_names(bits)))
+                    except Exception:
+                        pass
+                    time.sleep(self.INTERVAL_S)
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            return
+        try:
+            self.source = "nvidia-smi"
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
-                 "-i", str(self.gpu)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-i", str(self.device_index)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            self.source = None
 
-    def stop(self, t0: float | None = None, t1: float | None = None):
-        """Stop sampling; summarise the samples taken between host times t0 and t1."""
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        with open(self.path) as f:
-            lines = f.readlines()
-        os.unlink(self.path)
-        return summarize_clocks(lines, t0, t1)
+    def stop(self):
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(timeout=5)
+            self.thread = None
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            with open(self.path) as f:
+                self.rows = parse_smi_rows(f.readlines())
+            os.unlink(self.path)
+            self.proc = None
+
+    def window(self, t0: float | None = None, t1: float | None = None):
+        """Summary of the samples taken between host times t0 and t1."""
+        s = summarize_rows(self.rows, t0, t1)
+        if s is not None:
+            s["source"] = self.source
+        return s
 
 
-def summarize_clocks(lines, t0: float | None = None, t1: float | None = None):
-    """Median SM clock, max clock and active throttle reasons of nvidia-smi
-    CSV rows (the ClockSampler fields, no header, no units) whose timestamp
-    lies in [t0, t1] (host time); None if no row qualifies."""
+REASON_BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+
+def reason_names(bits: int) -> list:
+    """Names of the clock-event reasons set in an NVML reasons bitmask (the
+    ones that decide whether a timed run is kept)."""
+    return sorted(name for name, b in REASON_BITS.items() if bits & b)
+
+
+def parse_smi_rows(lines):
+    """nvidia-smi CSV rows (the ClockSampler fields, no header, no units) ->
+    (host time or None, sm MHz or None, max MHz or None, [active reasons])."""
     import datetime
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
     rows = []
     for line in lines:
         parts = [x.strip() for x in line.split(",")]
@@ -148,23 +239,33 @@ def summarize_clocks(lines, t0: float | None = None, t1: float | None = None):
             ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
         except ValueError:
             ts = None
-        if t0 is not None and ts is not None and not (t0 <= ts <= t1):
-            continue
-        rows.append(parts)
-    if not rows:
-        return None
 
-    def num(x):
-        try:
-            return float(x)
-        except ValueError:
-            return None
-    sm = [num(r[1]) for r in rows if num(r[1]) is not None]
-    mx = [num(r[2]) for r in rows if num(r[2]) is not None]
-    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-    reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        reasons = [names[i] for i in range(4) if parts[5 + i].lower().startswith("active")]
+        rows.append((ts, num(parts[1]), num(parts[2]), reasons))
+    return rows
+
+
+def summarize_rows(rows, t0: float | None = None, t1: float | None = None):
+    """Median SM clock, max clock and active reasons of the sample rows whose
+    time lies in [t0, t1]; None if no row qualifies."""
+    sel = [r for r in rows if t0 is None or r[0] is None or t0 <= r[0] <= t1]
+    if not sel:
+        return None
+    sm = [r[1] for r in sel if r[1] is not None]
+    mx = [r[2] for r in sel if r[2] is not None]
+    reasons = sorted({x for r in sel for x in r[3]})
     return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-            "reasons": reasons, "samples": len(rows)}
+            "reasons": reasons, "samples": len(sel)}
+
+
+def summarize_clocks(lines, t0: float | None = None, t1: float | None = None):
+    """summarize_rows over nvidia-smi CSV lines."""
+    return summarize_rows(parse_smi_rows(lines), t0, t1)
 
 
 def traffic_for(kernel_src: str, workload: str):
@@ -200,6 +301,182 @@ class L2Flush:
         self.r.sum()
 
 
+def roofline(kernel: str, bound: str, amount: float, ms: float, peaks: dict, peak_src: str,
+             sustained: bool = False, traffic=None) -> dict:
+    """Roofline record: `amount` algorithmic bytes (bound "hbm") or FLOPs
+    (bound "tensor") per launch over `ms` milliseconds, against the measured
+    HBM copy bandwidth or bf16 dense throughput (burst for a kernel timed by
+    itself, sustained for one timed inside a long run)."""
+    if bound == "hbm":
+        ach = amount / (ms * 1e-3) / 1e9
+        peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        unit, label = "GB/s", "HBM copy"
+    else:
+        ach = amount / (ms * 1e-3) / 1e12
+        key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+        peak = float(peaks.get(key, FALLBACK_PEAKS[key]))
+        unit, label = "TFLOP/s", "bf16 dense " + ("(sustained)" if sustained else "(burst)")
+    return {"kernel": kernel, "bound": bound, "achieved": round(ach, 2), "peak": peak, "unit": unit,
+            "frac": round(ach / peak, 4), "peak_source": f"{peak_src} {label}",
+            ("algorithmic_bytes" if bound == "hbm" else "algorithmic_flop"): amount, "ms": round(ms, 4),
+            "traffic": traffic}
+
+
+def timed_ms(fn, iters, flush, stream):
+    """Median device time (ms) of fn over `iters` calls, L2 flushed before
+    each, CUDA events on the launching stream."""
+    import torch
+    ts = []
+    for i in range(iters):
+        flush(i)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def fill_cache(pf, wl, d, dev, layers=1, sink_rope_in_attention=False):
+    """A cache holding d's sink, mid pool and recent blocks in every layer."""
+    cache = pf.PackedKVCache(pf.config_for(wl, layers=layers, sink_rope_in_attention=sink_rope_in_attention),
+                             device=dev)
+    for l in range(layers):
+        for s_ in range(wl.sink_blocks):
+            cache.append_block(l, d["sink_K"][:, s_].contiguous(), d["sink_V"][:, s_].contiguous())
+        if wl.pool_blocks:
+            cache.load_mid(l, d["mid_K"].contiguous(), d["mid_V"].contiguous())
+        for r in range(wl.recent_blocks):
+            cache.append_block(l, d["recent_K"][:, r].contiguous(), d["recent_V"][:, r].contiguous(),
+                               d["recent_Kc"][:, r].contiguous(), d["recent_Vc"][:, r].contiguous())
+    return cache
+
+
+def measure_stress(pf, synth, dev, flush, stream, peaks, src, iters) -> dict:
+    """The batch-2 stress layers (1,000-block compressed pool): selection,
+    the RoPE shift of every cached key and of the sink, attention with 16 and
+    64 routed blocks, and the allocation-free selection streaming the pool."""
+    import torch
+    out = {}
+    for name in ("stress16", "stress64"):
+        wl = synth.WORKLOADS[name]
+        d = synth.make_layer(wl, synth.nominal_seed(list(synth.WORKLOADS).index(name)), device=dev)
+        cache = fill_cache(pf, wl, d, dev)
+        B, H, D, n, nc, P = wl.batch, wl.heads, wl.head_dim, wl.n, wl.n_c, wl.pool_blocks
+        row = H * D * 2
+        r = {}
+        if name == "stress16":
+            ms = timed_ms(lambda: cache.select_mid(0, d["Q"]), iters, flush, stream)
+            # reads: the queries (bf16) and every live block's cached mean key (fp32)
+            r["select"] = roofline("qpool_kernel + score_mean_kernel", "hbm", B * n * row + B * P * H * D * 4, ms,
+                                   peaks, src)
+            info = cache.info(0)
+            sel = torch.empty((B, wl.n_top), dtype=torch.int32, device=dev)
+            ms = timed_ms(lambda: pf.pf_select_mid_static(d["Q"], B, n, H, info["pool_k"], info["pool_slots"], nc,
+                                                          info["mid_head"], P, wl.n_top, sel),
+                          iters, flush, stream)
+            # reads: the queries and every live block's n_c compressed keys
+            r["select_streaming"] = roofline("qpool_kernel + score_kernel", "hbm", B * n * row + B * P * nc * row,
+                                             ms, peaks, src)
+            parts = pf.PART_SINK | pf.PART_MID | pf.PART_RECENT
+            rows = B * (wl.sink_blocks * n + P * nc + wl.recent_blocks * (n + nc))
+            ms = timed_ms(lambda: cache.rope_shift(0, parts, 4), iters, flush, stream)
+            # 22 rotary pairs = 88 bytes read and 88 written per (key, head)
+            r["rope_shift_all"] = roofline("rope_shift_tma_kernel", "hbm", rows * H * 176, ms, peaks, src)
+            ms = timed_ms(lambda: cache.rope_shift(0, pf.PART_SINK, 4), iters, flush, stream)
+            r["rope_shift_sink"] = roofline("rope_shift_tma_kernel", "hbm", B * wl.sink_blocks * n * H * 176, ms,
+                                            peaks, src)
+        cache.select_mid(0, d["Q"])
+        O = torch.empty_like(d["Q"])
+        Lk = cache.info(0)["context_tokens"]
+        ms = timed_ms(lambda: cache.attend(0, d["Q"], d["K_cur"], d["V_cur"], O), iters, flush, stream)
+        r["attend"] = roofline("attend_kernel", "tensor", attention_flops(B, H, n, Lk, D), ms, peaks, src)
+        r["context_tokens"] = Lk
+        cache.poll_device_error()
+        out[name] = r
+        del cache, d, O
+        torch.cuda.empty_cache()
+    return out
+
+
+def measure_dense(pf, synth, dev, flush, stream, peaks, src, iters) -> dict:
+    """The dense layer: 6,240 queries over 748,800 full-resolution keys."""
+    import torch
+    wl = synth.WORKLOADS["dense"]
+    d = synth.make_layer(wl, synth.nominal_seed(list(synth.WORKLOADS).index("dense")), device=dev)
+    cache = fill_cache(pf, wl, d, dev)
+    O = torch.empty_like(d["Q"])
+    Lk = cache.info(0)["context_tokens"]
+    ms = timed_ms(lambda: cache.attend(0, d["Q"], d["K_cur"], d["V_cur"], O), iters, flush, stream)
+    r = {"context_tokens": Lk,
+         "attend": roofline("attend_kernel", "tensor", attention_flops(wl.batch, wl.heads, wl.n, Lk), ms, peaks, src)}
+    cache.poll_device_error()
+    del cache, d, O
+    torch.cuda.empty_cache()
+    return r
+
+
+def measure_block(pf, synth, dev, flush, stream, peaks, src, blocks=3) -> dict:
+    """One generated block of the 30-layer model at CFG batch 2 (cond +
+    uncond): 4 denoising steps x 30 layers of pf_attend_step (selection at
+    the first step, reused by the other three), then pf_finish_block (append
+    the block to every layer, evict the oldest compressed block, shift every
+    sink).  116-block pool per layer."""
+    import torch
+    wl = synth.WORKLOADS["step30"].replace(batch=2)
+    L, S = wl.layers, 4
+    B, H, D, n, nc = wl.batch, wl.heads, wl.head_dim, wl.n, wl.n_c
+    cache = pf.PackedKVCache(pf.config_for(wl, layers=L), device=dev)
+    blk = synth.make_block(wl, 77, dev)
+    pool = synth.bf16_normal((B, wl.pool_blocks, nc, H, D), 78, dev)
+    for l in range(L):
+        for _ in range(wl.sink_blocks):
+            cache.append_block(l, blk["K"], blk["V"])
+        cache.load_mid(l, pool, pool)
+        cache.append_block(l, blk["K"], blk["V"], blk["Kc"], blk["Vc"])
+    del pool
+    Qs = [synth.bf16_normal((B, n, H, D), 100 + l, dev) for l in range(L)]
+    Ks = [synth.bf16_normal((B, n, H, D), 200 + l, dev) for l in range(L)]
+    Vs = [synth.bf16_normal((B, n, H, D), 300 + l, dev) for l in range(L)]
+    Kcs = [synth.bf16_normal((B, nc, H, D), 400 + l, dev) for l in range(L)]
+    O = torch.empty_like(Qs[0])
+
+    def block():
+        for step in range(S):
+            for l in range(L):
+                cache.attend_step(l, step, Qs[l], Ks[l], Vs[l], O)
+        cache.finish_block(Ks, Vs, Kcs, Kcs)
+
+    block()
+    ms = timed_ms(block, blocks, flush, stream)
+    Lk = cache.info(0)["context_tokens"]
+    flops = L * S * attention_flops(B, H, n, Lk, D)
+    cache.poll_device_error()
+    r = {"ms_per_block": round(ms, 3), "layer_step_ms": round(ms / (L * S), 4), "context_tokens": Lk,
+         "attention_flop_per_block": flops,
+         # attend per layer and step; qpool + score_mean per layer at step 0;
+         # copy + key mean per layer's append; one shift launch for all sinks
+         "launches_per_block": L * S + 2 * L + 2 * L + 1,
+         "attend_block": roofline("attend_kernel (whole block: selection, appends and shifts included)", "tensor",
+                                  flops, ms, peaks, src, sustained=True)}
+    del cache, Qs, Ks, Vs, Kcs, O, blk
+    torch.cuda.empty_cache()
+    return r
+
+
+def measure_configs(which, pf, synth, dev, flush, stream, peaks, src, iters) -> dict:
+    """The workloads beside the headline, keyed by the configuration they stand for."""
+    out = {}
+    if "c2" in which:
+        out["c2_block_30_layers_4_steps_cfg2"] = measure_block(pf, synth, dev, flush, stream, peaks, src)
+    if "c3" in which:
+        out["c3_dense_748800_keys"] = measure_dense(pf, synth, dev, flush, stream, peaks, src, max(3, iters // 4))
+    if "c4" in which:
+        out.update({f"c4_{k}": v for k, v in measure_stress(pf, synth, dev, flush, stream, peaks, src, iters).items()})
+    return out
+
+
 def run_gpu(args):
     import torch
 
@@ -213,18 +490,28 @@ def run_gpu(args):
     dist_init("nccl")
     dev = torch.device("cuda", local)
     wl = synth.WORKLOADS[WORKLOAD]
+    H_all = wl.heads
+    sharded = args.shard == "heads"
+    base_seed = synth.nominal_seed(list(synth.WORKLOADS).index(WORKLOAD))
+    if sharded:
+        # one layer spread over the ranks by heads: every rank draws the same
+        # layer and keeps its own heads
+        lo, hi = head_shard(H_all, world, rank)
+        if hi <= lo:
+            raise SystemExit(f"--shard heads needs at most {H_all} ranks")
+        seed = base_seed
+        full = synth.make_layer(wl, seed, device=dev)
+        d = {k: (v[..., lo:hi, :].contiguous() if torch.is_tensor(v) and v.dim() >= 4 else v)
+             for k, v in full.items()}
+        del full
+        wl = wl.replace(heads=hi - lo)
+    else:
+        seed = rank_seed(base_seed, rank)
+        d = synth.make_layer(wl, seed, device=dev)
     B, H, D, n, nc = wl.batch, wl.heads, wl.head_dim, wl.n, wl.n_c
-    seed = rank_seed(synth.nominal_seed(list(synth.WORKLOADS).index(WORKLOAD)), rank)
-    d = synth.make_layer(wl, seed, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    cache = pf.PackedKVCache(pf.config_for(wl, layers=1), device=dev)
-    for s in range(wl.sink_blocks):
-        cache.append_block(0, d["sink_K"][:, s].contiguous(), d["sink_V"][:, s].contiguous())
-    cache.load_mid(0, d["mid_K"].contiguous(), d["mid_V"].contiguous())
-    for r in range(wl.recent_blocks):
-        cache.append_block(0, d["recent_K"][:, r].contiguous(), d["recent_V"][:, r].contiguous(),
-                           d["recent_Kc"][:, r].contiguous(), d["recent_Vc"][:, r].contiguous())
+    cache = fill_cache(pf, wl, d, dev)
     # the current block's inputs (resident); its compressed copy for the append
     Q, Kn, Vn = d["Q"], d["K_cur"], d["V_cur"]
     Kcn = synth.bf16_normal((B, nc, H, D), seed + 1, dev)
@@ -232,12 +519,25 @@ def run_gpu(args):
     O = torch.empty_like(Q)
     info0 = cache.info(0)
     Lk = info0["context_tokens"]
-    flops = attention_flops(B, H, n, Lk, D)
+    flops = attention_flops(B, H, n, Lk, D)              # this rank's heads
+    # [B, live blocks] partial (then summed) block scores of the sharded selection;
+    # the pool stays full from step to step (each append evicts one block)
+    scores = torch.zeros((B, max(1, info0["mid_count"])), dtype=torch.float32, device=dev)
+    import torch.distributed as dist
 
-    ev_att = []
+    def all_reduce_sum(t):
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.SUM)
+
+    def select(q):
+        if sharded:
+            select_head_sharded(cache, 0, q, scores, H_all, all_reduce_sum, pf.ROUTE_SCORES_ONLY, pf.ROUTE_GIVEN)
+            return 3
+        cache.select_mid(0, q)
+        return 2
 
     def step(q, k, v, kc, vc, out, att_events=None):
-        cache.select_mid(0, q)
+        nl = select(q)
         if att_events is not None:
             att_events[0].record(stream)
         cache.attend(0, q, k, v, out)
@@ -246,10 +546,11 @@ def run_gpu(args):
         ev = cache.append_block(0, k, v, kc, vc)
         if ev:
             cache.rope_shift(0, pf.PART_SINK, ev * wl.block_frames)
-        return LAUNCHES_PER_STEP_BASE + (1 if ev else 0)
+        return LAUNCHES_PER_STEP_BASE - 2 + nl + (1 if ev else 0)
 
     clocks = ClockSampler(local)
     clocks.start()
+    t_run0 = time.time()
     flush = L2Flush(dev)
     for i in range(args.warmup):
         flush(i)
@@ -274,14 +575,15 @@ def run_gpu(args):
     torch.cuda.synchronize(dev)
     t_end = time.time()
     barrier()
-    clk = clocks.stop(t_start, t_end)
     cache.poll_device_error()
     step_ms = [a.elapsed_time(b) for a, b in ev_step]
     att_ms = [a.elapsed_time(b) for a, b in ev_att]
     total_ms = reduce_max(sum(step_ms), dev)
     att_mean_ms = reduce_max(statistics.mean(att_ms), dev)
     ms_per_step = total_ms / args.steps
-    value = world * args.steps * flops / (total_ms * 1e-3) / 1e12
+    # whole-job work: every rank's heads (sharded: one layer; replicas: one layer each)
+    job_flops = attention_flops(B, H_all, n, Lk, D) if sharded else world * flops
+    value = args.steps * job_flops / (total_ms * 1e-3) / 1e12
 
     # ---- end to end through the public API with host buffers.  Each step's
     # inputs come from pinned host memory and its output goes back to pinned
@@ -342,12 +644,21 @@ def run_gpu(args):
     torch.cuda.synchronize(dev)
     barrier()
     e2e_ms = reduce_max(e0.elapsed_time(e1), dev)
-    e2e_value = world * args.steps * flops / (e2e_ms * 1e-3) / 1e12
+    e2e_value = args.steps * job_flops / (e2e_ms * 1e-3) / 1e12
     cache.poll_device_error()
+    cache.close()
+    del cache, din, dO, hin, hO
+    torch.cuda.empty_cache()
 
     peaks, peak_src = load_peaks()
-    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    achieved = flops / (att_mean_ms * 1e-3) / 1e12
+    configs = {}
+    if rank == 0 and args.configs != "none":
+        which = {"c2", "c3", "c4"} if args.configs == "all" else set(args.configs.split(","))
+        configs = measure_configs(which, pf, synth, dev, flush, stream, peaks, peak_src, max(args.steps, 5))
+    t_run1 = time.time()
+    clocks.stop()
+    att = roofline("attend_kernel", "tensor", flops, att_mean_ms, peaks, peak_src,
+                   traffic=traffic_for(os.path.join(ROOT, "packed_kv_cache_b200", "csrc", "attend.cu"), WORKLOAD))
     line = {
         "metric": "packed-cache attention TFLOP/s (per-layer step)",
         "value": round(value, 2),
@@ -357,7 +668,7 @@ def run_gpu(args):
         "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if sharded else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
@@ -366,29 +677,23 @@ def run_gpu(args):
                          "compressed 182 tokens/block, pool 40, top-16, context 27872 keys; "
                          "step = select + attend + append(evict) + sink RoPE shift"),
             "context_tokens": Lk,
-            "attention_flop_per_step": flops,
+            "attention_flop_per_step": job_flops,
             "l2": "flushed between steps (256 MB write, then 256 MB read of another buffer), outside the step events",
-            "parallelism": f"replicas x{world} (independent streams, no collective)",
+            "parallelism": (f"heads sharded x{world} ({H} of {H_all} heads on this rank; NCCL all-reduce of the "
+                            f"[B, P] partial block scores before the top-k)" if sharded else
+                            f"replicas x{world} (independent streams, no collective)"),
         },
         "attention_ms": round(att_mean_ms, 4),
-        "roofline": {
-            "kernel": "attend_kernel",
-            "bound": "tensor",
-            "achieved": round(achieved, 2),
-            "peak": peak,
-            "unit": "TFLOP/s",
-            "frac": round(achieved / peak, 4),
-            "peak_source": f"{peak_src} bf16 dense (burst)",
-            "traffic": traffic_for(os.path.join(ROOT, "packed_kv_cache_b200", "csrc", "attend.cu"), WORKLOAD),
-        },
+        "roofline": att,
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / args.steps, 4)},
         "gpu_launches": launches,
-        "clocks": clk,
+        "clocks": clocks.window(t_start, t_end),
+        "clocks_run": clocks.window(t_run0, t_run1),
+        "configs": configs,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:   # the oracle's timing: one process only
-        line["cpu_baseline"] = cpu_baseline(d, wl, budget_s=args.cpu_seconds)
-    cache.close()
+        line["cpu_baseline"] = cpu_baseline({k: v for k, v in d.items()}, wl, budget_s=args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
     import torch.distributed as dist
@@ -527,28 +832,10 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-# ---------------------------------------------------------------- per-kernel suite
-
-def _timed(fn, iters, flush, stream):
-    """Median device time (ms) of fn over iters calls, L2 flushed before each."""
-    import torch
-    ts = []
-    for i in range(iters):
-        flush(i)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        fn()
-        b.record(stream)
-        torch.cuda.synchronize()
-        ts.append(a.elapsed_time(b))
-    return statistics.median(ts)
-
+# ---------------------------------------------------------------- configs only
 
 def run_suite(args):
-    """One JSON line per hot-path kernel on the workload its roofline is
-    measured on: scoring and RoPE shift on the batch-2, 1,000-block stress
-    layer (HBM-bound), attention on the layer / stress / dense workloads
-    (tensor-bound), append, and the 30-layer block step."""
+    """The extra configurations alone (no headline), one JSON line each."""
     import torch
 
     import synth
@@ -560,145 +847,14 @@ def run_suite(args):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     peaks, src = load_peaks()
-    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    tfl = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    flush = L2Flush(dev)
-    iters = max(args.steps, 5)
-    out = []
-
-    def build(wl, d, sink_rope_in_attention=False):
-        cache = pf.PackedKVCache(pf.config_for(wl, layers=1, sink_rope_in_attention=sink_rope_in_attention),
-                                 device=dev)
-        for s_ in range(wl.sink_blocks):
-            cache.append_block(0, d["sink_K"][:, s_].contiguous(), d["sink_V"][:, s_].contiguous())
-        if wl.pool_blocks:
-            cache.load_mid(0, d["mid_K"].contiguous(), d["mid_V"].contiguous())
-        for r in range(wl.recent_blocks):
-            cache.append_block(0, d["recent_K"][:, r].contiguous(), d["recent_V"][:, r].contiguous(),
-                               d["recent_Kc"][:, r].contiguous(), d["recent_Vc"][:, r].contiguous())
-        return cache
-
-    def line(kernel, workload, ms, bound, amount, unit_amount):
-        if bound == "hbm":
-            ach = amount / (ms * 1e-3) / 1e9
-            return {"kernel": kernel, "workload": workload, "ms": round(ms, 4), "bound": "hbm",
-                    "algorithmic_bytes": amount, "achieved": round(ach, 1), "unit": "GB/s", "peak": hbm,
-                    "frac": round(ach / hbm, 4), "peak_source": f"{src} HBM copy"}
-        ach = amount / (ms * 1e-3) / 1e12
-        return {"kernel": kernel, "workload": workload, "ms": round(ms, 4), "bound": "tensor",
-                "algorithmic_flop": amount, "achieved": round(ach, 1), "unit": "TFLOP/s", "peak": tfl,
-                "frac": round(ach / tfl, 4), "peak_source": f"{src} bf16 dense (burst)"}
-
-    want = lambda part: args.only in ("all", part)  # noqa: E731
-
-    if want("stress") or args.only == "stress16":
-        # ---- stress layers: selection and RoPE shift (HBM), attention
-        for name in ("stress16",) if args.only == "stress16" else ("stress16", "stress64"):
-            wl = synth.WORKLOADS[name]
-            d = synth.make_layer(wl, synth.nominal_seed(list(synth.WORKLOADS).index(name)), device=dev)
-            cache = build(wl, d)
-            B, H, D, n, nc, P = wl.batch, wl.heads, wl.head_dim, wl.n, wl.n_c, wl.pool_blocks
-            row = H * D * 2
-            if name == "stress16":
-                ms = _timed(lambda: cache.select_mid(0, d["Q"]), iters, flush, stream)
-                # reads: the queries (bf16) and each block's cached mean key (fp32)
-                out.append(line("select (qpool + mean-key scores + top-k)", name, ms, "hbm",
-                                B * n * row + B * P * H * D * 4, None))
-                parts = pf.PART_SINK | pf.PART_MID | pf.PART_RECENT
-                ms = _timed(lambda: cache.rope_shift(0, parts, 4), iters, flush, stream)
-                rows = B * (wl.sink_blocks * n + P * nc + wl.recent_blocks * (n + nc))
-                out.append(line("rope_shift (sink + mid + recent)", name, ms, "hbm", rows * H * 176, None))
-                rows_sink = B * wl.sink_blocks * n
-                ms = _timed(lambda: cache.rope_shift(0, pf.PART_SINK, 4), iters, flush, stream)
-                out.append(line("rope_shift (sink)", name, ms, "hbm", rows_sink * H * 176, None))
-            cache.select_mid(0, d["Q"])
-            O = torch.empty_like(d["Q"])
-            Lk = cache.info(0)["context_tokens"]
-            ms = _timed(lambda: cache.attend(0, d["Q"], d["K_cur"], d["V_cur"], O), iters, flush, stream)
-            out.append(line("attend", f"{name} (Lk {Lk})", ms, "tensor", attention_flops(B, H, n, Lk, D), None))
-            cache.poll_device_error()
-            del cache, d
-            torch.cuda.empty_cache()
-
-    if want("layer"):
-        # ---- pages-scale layer: append (HBM) and attention
-        wl = synth.WORKLOADS["layer"]
-        d = synth.make_layer(wl, synth.nominal_seed(1), device=dev)
-        cache = build(wl, d)
-        B, H, D, n, nc = wl.batch, wl.heads, wl.head_dim, wl.n, wl.n_c
-        row = H * D * 2
-        Kc = synth.bf16_normal((B, nc, H, D), 5, dev)
-        ms = _timed(lambda: cache.append_block(0, d["K_cur"], d["V_cur"], Kc, Kc), iters, flush, stream)
-        out.append(line("append (copy)", "layer", ms, "hbm", 2 * 2 * B * (n + nc) * row, None))
-        cache.select_mid(0, d["Q"])
-        O = torch.empty_like(d["Q"])
-        Lk = cache.info(0)["context_tokens"]
-        ms = _timed(lambda: cache.attend(0, d["Q"], d["K_cur"], d["V_cur"], O), iters, flush, stream)
-        out.append(line("attend", f"layer (Lk {Lk})", ms, "tensor", attention_flops(B, H, n, Lk, D), None))
-        cache.poll_device_error()
-        del cache
-        torch.cuda.empty_cache()
-        # the sink's RoPE shift applied inside attention (sink K tiles rotated
-        # in shared memory); the in-place shift pass disappears from the step
-        cache = build(wl, d, sink_rope_in_attention=True)
-        cache.rope_shift(0, pf.PART_SINK, 4)
-        cache.select_mid(0, d["Q"])
-        ms = _timed(lambda: cache.attend(0, d["Q"], d["K_cur"], d["V_cur"], O), iters, flush, stream)
-        out.append(line("attend, sink RoPE shift applied in attention", f"layer (Lk {Lk})", ms, "tensor",
-                        attention_flops(B, H, n, Lk, D), None))
-        cache.poll_device_error()
-        del cache
-        torch.cuda.empty_cache()
-
-    if want("dense"):
-        # ---- dense 748,800-key layer
-        wl = synth.WORKLOADS["dense"]
-        d = synth.make_layer(wl, synth.nominal_seed(3), device=dev)
-        cache = build(wl, d)
-        O = torch.empty_like(d["Q"])
-        Lk = cache.info(0)["context_tokens"]
-        ms = _timed(lambda: cache.attend(0, d["Q"], d["K_cur"], d["V_cur"], O), max(3, iters // 4), flush, stream)
-        out.append(line("attend", f"dense (Lk {Lk})", ms, "tensor", attention_flops(1, wl.heads, wl.n, Lk), None))
-        cache.poll_device_error()
-        del cache, d
-        torch.cuda.empty_cache()
-
-    if want("step30"):
-        # ---- the 30-layer block step: per layer select, attend, append; then the sink shift of all layers
-        wl = synth.WORKLOADS["step30"]
-        L = wl.layers
-        cache = pf.PackedKVCache(pf.config_for(wl, layers=L), device=dev)
-        B, H, D, n, nc = wl.batch, wl.heads, wl.head_dim, wl.n, wl.n_c
-        blk = synth.make_block(wl, 77, dev)
-        pool = synth.bf16_normal((B, wl.pool_blocks, nc, H, D), 78, dev)
-        for l in range(L):
-            for _ in range(wl.sink_blocks):
-                cache.append_block(l, blk["K"], blk["V"])
-            cache.load_mid(l, pool, pool)
-            cache.append_block(l, blk["K"], blk["V"], blk["Kc"], blk["Vc"])
-        Qs = [synth.bf16_normal((B, n, H, D), 100 + l, dev) for l in range(L)]
-        O = torch.empty_like(Qs[0])
-
-        def block_step():
-            ev = 0
-            for l in range(L):
-                cache.select_mid(l, Qs[l])
-                cache.attend(l, Qs[l], blk["K"], blk["V"], O)
-                ev = cache.append_block(l, blk["K"], blk["V"], blk["Kc"], blk["Vc"])
-            if ev:
-                cache.rope_shift(-1, pf.PART_SINK, ev * wl.block_frames)
-
-        for _ in range(2):
-            block_step()
-        ms = _timed(block_step, 5, flush, stream)
-        Lk = cache.info(0)["context_tokens"]
-        st = line("30-layer block step", f"step30 (30 layers, pool {wl.pool_blocks}, Lk {Lk})", ms, "tensor",
-                  L * attention_flops(B, H, n, Lk, D), None)
-        st["layer_step_ms"] = round(ms / L, 4)
-        out.append(st)
-        cache.poll_device_error()
-    for o in out:
-        print(json.dumps(o), flush=True)
+    which = {"c2", "c3", "c4"} if args.configs in ("all", "none") else set(args.configs.split(","))
+    clocks = ClockSampler(0)
+    clocks.start()
+    out = measure_configs(which, pf, synth, dev, L2Flush(dev), stream, peaks, src, max(args.steps, 5))
+    clocks.stop()
+    for k, v in out.items():
+        print(json.dumps({"config": k, **v}), flush=True)
+    print(json.dumps({"clocks": clocks.window()}), flush=True)
 
 
 def main(argv=None):
@@ -713,11 +869,14 @@ def main(argv=None):
                     help="reference arm: host seconds for the warm-up and timed steps together")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--configs", default="all",
+                    help="workloads measured beside the headline: all, none, or a comma list of c2 (30-layer "
+                         "block, 4 denoising steps, CFG batch 2), c3 (dense layer), c4 (stress layers)")
     ap.add_argument("--suite", action="store_true",
-                    help="one JSON line per hot-path kernel on its roofline workload (not the headline line)")
-    ap.add_argument("--only", default="all",
-                    help="suite part: all, stress (selection, RoPE, attention on the stress layers), "
-                         "stress16 (the batch-2 stress layer only), layer, dense, step30")
+                    help="only the --configs workloads, one JSON line each (no headline)")
+    ap.add_argument("--shard", default="none", choices=["none", "heads"],
+                    help="heads: one layer spread over the ranks by heads (strong scaling; one NCCL all-reduce "
+                         "of the partial block scores per step); none: independent replicas (weak scaling)")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)   # at least 3 untimed warm-up steps
     if args.impl == "reference":
