@@ -188,7 +188,7 @@ pf_status pf_cache_load_mid(pf_cache* cache, int layer, const void* Kc, const vo
  * sel_out (optional, device, [B, min(n_top, mid_count)] int32): the chosen
  * blocks by age (0 = oldest live block), ascending.
  * scores_out (optional, device, [B, mid_count] float): S by age.
- * Two kernel launches; no host synchronisation.
+ * One kernel launch; no host synchronisation.
  */
 pf_status pf_select_mid(pf_cache* cache, int layer, const void* Q, int32_t* sel_out,
                         float* scores_out, void* stream);
@@ -232,9 +232,8 @@ typedef struct pf_select_opts {
  * pf_select_mid with a routing policy (see above).  opts NULL = the method's
  * defaults (PF_ROUTE_SCORE, every query row, every head) = pf_select_mid.
  * sel_out / scores_out as for pf_select_mid (scores_out is required for
- * PF_ROUTE_SCORES_ONLY and ignored by PF_ROUTE_FIFO).  PF_ROUTE_SCORE and
- * PF_ROUTE_SCORES_ONLY launch two kernels, PF_ROUTE_GIVEN and PF_ROUTE_FIFO
- * one.  Errors: PF_ERR_ARG for a bad policy, stride, head range, or a
+ * PF_ROUTE_SCORES_ONLY and ignored by PF_ROUTE_FIFO).  Every policy
+ * launches one kernel.  Errors: PF_ERR_ARG for a bad policy, stride, head range, or a
  * missing scores_in / scores_out.
  */
 pf_status pf_select_mid_ex(pf_cache* cache, int layer, const void* Q, const pf_select_opts* opts,
@@ -345,8 +344,9 @@ pf_status pf_finish_block(pf_cache* cache, const void* const* K, const void* con
  * The first call on a device looks up the array's device address with that
  * device current (make that first call before any stream capture); the
  * address is kept for the process, so a cudaDeviceReset of that device
- * leaves it stale (do not call this again on a device after resetting it).  Every
- * call clears what must start at zero and then shares the one array: calls
+ * leaves it stale (do not call this again on a device after resetting
+ * it).  Every call clears what must start at zero and then shares the one
+ * array: calls
  * that overlap on the GPU (different streams, or different host threads,
  * on one device) race and must not be made.  Three launches on `stream`
  * (one memset, two kernels); no host synchronisation.
