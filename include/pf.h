@@ -309,6 +309,32 @@ pf_status pf_finish_block(pf_cache* cache, const void* const* K, const void* con
                           const void* const* Kc, const void* const* Vc, int* evicted, void* stream);
 
 /*
+ * Saving and restoring a cache.  Everything on the device (every partition,
+ * the pool's mean keys, each layer's stored selection) lives in the
+ * caller's arena; the library's only other state is small host state per
+ * layer (ring heads and counts, blocks seen and evicted, accumulated sink
+ * shift, selection validity).  To save a cache: copy its arena (after its
+ * stream's work is done) and pf_cache_save_state.  To restore: create a
+ * cache with the same configuration, copy the saved arena into the new
+ * arena (after pf_cache_create's clearing, on the same stream or after it),
+ * then pf_cache_load_state.  (Not a step of the method: an interface of
+ * this library.)
+ *
+ * pf_cache_state_bytes: bytes of the saved host state (a header with the
+ * configuration, then one record per layer).
+ * pf_cache_save_state: write it into `buf` (host memory, `bytes` >= the
+ * size; PF_ERR_ARG otherwise).
+ * pf_cache_load_state: replace the cache's host state by a saved one.
+ * PF_ERR_ARG if `buf` is not a saved state of this size and version;
+ * PF_ERR_STATE if it was saved from a cache with another configuration or
+ * holds counts outside the configuration's limits (the cache is then left
+ * unchanged).  Launches nothing.
+ */
+pf_status pf_cache_state_bytes(const pf_cache* cache, size_t* bytes);
+pf_status pf_cache_save_state(const pf_cache* cache, void* buf, size_t bytes);
+pf_status pf_cache_load_state(pf_cache* cache, const void* buf, size_t bytes);
+
+/*
  * Limits of pf_select_mid_static (its scratch is a fixed array in the library).
  */
 #define PF_STATIC_MAX_BATCH 8

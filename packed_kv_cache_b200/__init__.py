@@ -22,6 +22,7 @@ __all__ = [
     "pf_cache_layer_info", "pf_cache_append_block", "pf_cache_load_mid", "pf_select_mid",
     "pf_rope_shift", "pf_attend", "pf_poll_device_error", "pf_selftest_wait_timeout",
     "pf_select_mid_static", "pf_select_mid_ex", "SelectOpts", "pf_attend_step", "pf_finish_block",
+    "pf_cache_state_bytes", "pf_cache_save_state", "pf_cache_load_state",
     "ROUTE_SCORE", "ROUTE_SCORES_ONLY", "ROUTE_GIVEN", "ROUTE_FIFO",
     "PackedKVCache", "config_for",
 ]
@@ -118,6 +119,9 @@ def _load():
         "pf_selftest_wait_timeout": ([vp, u32, vp], i32),
         "pf_select_mid_static": ([vp, i32, i32, i32, vp, i32, i32, i32, i32, i32, vp, vp, vp], i32),
         "pf_attend_step": ([vp, i32, i32, vp, vp, vp, vp, vp, vp], i32),
+        "pf_cache_state_bytes": ([vp, ctypes.POINTER(ctypes.c_size_t)], i32),
+        "pf_cache_save_state": ([vp, vp, ctypes.c_size_t], i32),
+        "pf_cache_load_state": ([vp, vp, ctypes.c_size_t], i32),
         "pf_finish_block": ([vp, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
                              ctypes.POINTER(vp), ctypes.POINTER(i32), vp], i32),
     }
@@ -306,6 +310,28 @@ def pf_finish_block(handle, K, V, Kc=None, Vc=None, stream=None) -> int:
     return ev.value
 
 
+def pf_cache_state_bytes(handle) -> int:
+    """Bytes of the cache's saved host state."""
+    out = ctypes.c_size_t()
+    _check("pf_cache_state_bytes", lib.pf_cache_state_bytes(handle, ctypes.byref(out)))
+    return out.value
+
+
+def pf_cache_save_state(handle) -> bytes:
+    """The cache's host state (ring heads, counts, shifts, selection validity)
+    as bytes; with a copy of the arena it restores the cache."""
+    n = pf_cache_state_bytes(handle)
+    buf = ctypes.create_string_buffer(n)
+    _check("pf_cache_save_state", lib.pf_cache_save_state(handle, buf, n))
+    return buf.raw
+
+
+def pf_cache_load_state(handle, state: bytes) -> None:
+    """Replace the cache's host state by a saved one (same configuration)."""
+    buf = ctypes.create_string_buffer(bytes(state), len(state))
+    _check("pf_cache_load_state", lib.pf_cache_load_state(handle, buf, len(state)))
+
+
 def pf_poll_device_error(handle, stream=None) -> int:
     """Synchronise `stream` and read (then clear) the cache's device error
     word; raises PF_ERR_TIMEOUT if a bounded wait gave up."""
@@ -456,6 +482,21 @@ class PackedKVCache:
             for t in ts:
                 _expect(t, name, torch.bfloat16, self._rows(rows))
         return pf_finish_block(self.handle, K, V, Kc, Vc, stream)
+
+    def save(self) -> tuple:
+        """(host state bytes, a device copy of the arena) after the current
+        stream's work; restore with PackedKVCache.restore."""
+        torch.cuda.current_stream(self.arena.device).synchronize()
+        return pf_cache_save_state(self.handle), self.arena.clone()
+
+    @classmethod
+    def restore(cls, cfg: Config, saved: tuple, device=None) -> "PackedKVCache":
+        """A new cache holding a saved one's contents (same configuration)."""
+        state, arena = saved
+        c = cls(cfg, device=device if device is not None else arena.device)
+        c.arena.copy_(arena)            # after the creation's clearing, on the same stream
+        pf_cache_load_state(c.handle, state)
+        return c
 
     def poll_device_error(self, stream=None) -> int:
         """See pf_poll_device_error."""

@@ -917,6 +917,103 @@ pf_status pf_finish_block(pf_cache* c, const void* const* K, const void* const* 
   return PF_OK;
 }
 
+// Saved host state: a header (magic, version, the configuration) and one
+// record per layer.
+namespace {
+constexpr uint32_t kStateMagic = 0x50465354u;   // "PFST"
+constexpr uint32_t kStateVersion = 1;
+struct StateHeader {
+  uint32_t magic, version;
+  pf_config cfg;
+};
+struct LayerState {
+  int32_t blocks_seen, sink_filled, recent_count, recent_head, mid_count, mid_head, sel_valid, n_sel;
+  int64_t evicted, total_shift;
+};
+}  // namespace
+
+pf_status pf_cache_state_bytes(const pf_cache* c, size_t* bytes) {
+  if (c == nullptr || bytes == nullptr) return fail(PF_ERR_ARG, "cache and bytes must not be NULL");
+  *bytes = sizeof(StateHeader) + sizeof(LayerState) * static_cast<size_t>(c->cfg.layers);
+  return PF_OK;
+}
+
+pf_status pf_cache_save_state(const pf_cache* c, void* buf, size_t bytes) {
+  size_t need = 0;
+  pf_status s = pf_cache_state_bytes(c, &need);
+  if (s != PF_OK) return s;
+  if (buf == nullptr || bytes < need) return fail(PF_ERR_ARG, "state buffer of %zu bytes, %zu needed", bytes, need);
+  StateHeader h;
+  std::memset(&h, 0, sizeof(h));
+  h.magic = kStateMagic;
+  h.version = kStateVersion;
+  h.cfg = c->cfg;
+  char* out = static_cast<char*>(buf);
+  std::memcpy(out, &h, sizeof(h));
+  out += sizeof(h);
+  for (const Layer& Ly : c->L) {
+    LayerState r;
+    std::memset(&r, 0, sizeof(r));
+    r.blocks_seen = Ly.blocks_seen;
+    r.sink_filled = Ly.sink_filled;
+    r.recent_count = Ly.recent_count;
+    r.recent_head = Ly.recent_head;
+    r.mid_count = Ly.mid_count;
+    r.mid_head = Ly.mid_head;
+    r.sel_valid = Ly.sel_valid ? 1 : 0;
+    r.n_sel = Ly.n_sel;
+    r.evicted = Ly.evicted;
+    r.total_shift = Ly.total_shift;
+    std::memcpy(out, &r, sizeof(r));
+    out += sizeof(r);
+  }
+  return PF_OK;
+}
+
+pf_status pf_cache_load_state(pf_cache* c, const void* buf, size_t bytes) {
+  size_t need = 0;
+  pf_status s = pf_cache_state_bytes(c, &need);
+  if (s != PF_OK) return s;
+  if (buf == nullptr || bytes != need) return fail(PF_ERR_ARG, "state of %zu bytes, %zu expected", bytes, need);
+  const char* in = static_cast<const char*>(buf);
+  StateHeader h;
+  std::memcpy(&h, in, sizeof(h));
+  in += sizeof(h);
+  if (h.magic != kStateMagic || h.version != kStateVersion) return fail(PF_ERR_ARG, "not a saved cache state");
+  if (std::memcmp(&h.cfg, &c->cfg, sizeof(pf_config)) != 0)
+    return fail(PF_ERR_STATE, "the state was saved from a cache with another configuration");
+  const pf_config& cf = c->cfg;
+  std::vector<LayerState> rs(static_cast<size_t>(cf.layers));
+  for (int l = 0; l < cf.layers; ++l) {
+    LayerState& r = rs[static_cast<size_t>(l)];
+    std::memcpy(&r, in, sizeof(r));
+    in += sizeof(r);
+    const int cap = cf.mid_capacity;
+    const bool okay = r.blocks_seen >= 0 && r.sink_filled >= 0 && r.sink_filled <= cf.sink_blocks &&
+                      r.recent_count >= 0 && r.recent_count <= cf.recent_blocks && r.recent_head >= 0 &&
+                      r.recent_head < cf.recent_blocks && r.mid_count >= 0 && r.mid_count <= cap &&
+                      r.mid_head >= 0 && r.mid_head < c->g.slots && (r.sel_valid == 0 || r.sel_valid == 1) &&
+                      r.n_sel >= 0 && r.n_sel <= cf.n_top && r.n_sel <= r.mid_count && r.evicted >= 0 &&
+                      (r.sink_filled == cf.sink_blocks || (r.recent_count == 0 && r.mid_count == 0));
+    if (!okay) return fail(PF_ERR_STATE, "layer %d of the saved state is outside the configuration's limits", l);
+  }
+  for (int l = 0; l < cf.layers; ++l) {
+    const LayerState& r = rs[static_cast<size_t>(l)];
+    Layer& Ly = c->L[l];
+    Ly.blocks_seen = r.blocks_seen;
+    Ly.sink_filled = r.sink_filled;
+    Ly.recent_count = r.recent_count;
+    Ly.recent_head = r.recent_head;
+    Ly.mid_count = r.mid_count;
+    Ly.mid_head = r.mid_head;
+    Ly.sel_valid = r.sel_valid != 0;
+    Ly.n_sel = r.n_sel;
+    Ly.evicted = r.evicted;
+    Ly.total_shift = r.total_shift;
+  }
+  return PF_OK;
+}
+
 pf_status pf_poll_device_error(pf_cache* c, void* stream, unsigned* code) {
   if (c == nullptr) return fail(PF_ERR_ARG, "cache is NULL");
   cudaStream_t st = static_cast<cudaStream_t>(stream);

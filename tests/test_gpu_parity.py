@@ -747,6 +747,58 @@ def test_sink_rope_in_attention_needs_a_full_sink(pf):
     assert cache.info(0)["total_shift"] == 4
 
 
+# ------------------------------------------------------------------ save and restore
+
+def test_save_and_restore_a_cache(pf):
+    # a cache restored from its saved host state and a copy of its arena
+    # behaves exactly as the original: same layer states, bit-identical
+    # attention with the stored selection, and the same evolution afterwards
+    L = 2
+    wl = _wl("ragged_a").replace(mid_capacity=3, n_top=2, planted=0, layers=L)
+    B, n, H, D = wl.batch, wl.n, wl.heads, wl.head_dim
+    cfg = pf.config_for(wl)
+    cache = pf.PackedKVCache(cfg)
+    for i in range(7):                                  # sink, recent, a full pool and two evictions
+        blks = [synth.make_block(wl, 500 + 10 * i + l) for l in range(L)]
+        cache.finish_block([b_["K"].cuda() for b_ in blks], [b_["V"].cuda() for b_ in blks],
+                           [b_["Kc"].cuda() for b_ in blks], [b_["Vc"].cuda() for b_ in blks])
+    Q = synth.bf16_normal((B, n, H, D), 600).cuda()
+    K = synth.bf16_normal((B, n, H, D), 601).cuda()
+    for l in range(L):
+        cache.attend_step(l, 0, Q, K, K)                # stores a selection in every layer
+    saved = cache.save()
+    twin = pf.PackedKVCache.restore(cfg, saved)
+    for l in range(L):
+        a, b = cache.info(l), twin.info(l)
+        for k in ("blocks_seen", "sink_filled", "recent_count", "recent_head", "mid_count", "mid_head",
+                  "selection_valid", "n_selected", "context_tokens", "evicted", "total_shift"):
+            assert a[k] == b[k], (l, k)
+        assert a["selection_valid"] == 1 and a["evicted"] >= 2
+        O1 = cache.attend_step(l, 1, Q, K, K)           # reuses the stored selection
+        O2 = twin.attend_step(l, 1, Q, K, K)
+        assert torch.equal(O1, O2)
+    blks = [synth.make_block(wl, 700 + l) for l in range(L)]
+    args = ([b_["K"].cuda() for b_ in blks], [b_["V"].cuda() for b_ in blks],
+            [b_["Kc"].cuda() for b_ in blks], [b_["Vc"].cuda() for b_ in blks])
+    assert cache.finish_block(*args) == twin.finish_block(*args) == 1
+    for l in range(L):
+        assert torch.equal(cache.attend_step(l, 0, Q, K, K), twin.attend_step(l, 0, Q, K, K))
+    # a state of another configuration, or not a state at all, is refused
+    other = pf.PackedKVCache(pf.config_for(wl.replace(n_top=1)))
+    with pytest.raises(pf.PFError) as e:
+        pf.pf_cache_load_state(other.handle, saved[0])
+    assert e.value.status_name == "PF_ERR_STATE"
+    with pytest.raises(pf.PFError) as e:
+        pf.pf_cache_load_state(twin.handle, b"\0" * len(saved[0]))
+    assert e.value.status_name == "PF_ERR_ARG"
+    bad = bytearray(saved[0])
+    # the last layer's record: eight int32 (mid_count the fifth) then two int64
+    bad[-32:-28] = (10 ** 6).to_bytes(4, "little")      # its mid_count far past the capacity
+    with pytest.raises(pf.PFError) as e:
+        pf.pf_cache_load_state(twin.handle, bytes(bad))
+    assert e.value.status_name == "PF_ERR_STATE"
+
+
 # ------------------------------------------------------------------ several devices
 
 def test_two_devices_in_one_process(pf):
