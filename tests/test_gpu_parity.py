@@ -758,7 +758,7 @@ def test_save_and_restore_a_cache(pf):
     B, n, H, D = wl.batch, wl.n, wl.heads, wl.head_dim
     cfg = pf.config_for(wl)
     cache = pf.PackedKVCache(cfg)
-    for i in range(7):                                  # sink, recent, a full pool and two evictions
+    for i in range(8):                                  # sink, recent, a full pool and two evictions
         blks = [synth.make_block(wl, 500 + 10 * i + l) for l in range(L)]
         cache.finish_block([b_["K"].cuda() for b_ in blks], [b_["V"].cuda() for b_ in blks],
                            [b_["Kc"].cuda() for b_ in blks], [b_["Vc"].cuda() for b_ in blks])
