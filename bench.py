@@ -49,9 +49,9 @@ sys.path.insert(0, ROOT)
 
 WORKLOAD = "layer"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# library kernels per step: qpool + score_mean (select), attend, copy_runs +
-# kmean (append with a compressed copy), and rope_shift when a block was evicted
-LAUNCHES_PER_STEP_BASE = 5
+# library kernels per step besides the selection's: attend, copy_runs + kmean
+# (append with a compressed copy); rope_shift is added when a block was evicted
+LAUNCHES_PER_STEP_BASE = 3
 
 
 # ---------------------------------------------------------------- distributed plumbing
@@ -369,7 +369,7 @@ def measure_stress(pf, synth, dev, flush, stream, peaks, src, iters) -> dict:
         if name == "stress16":
             ms = timed_ms(lambda: cache.select_mid(0, d["Q"]), iters, flush, stream)
             # reads: the queries (bf16) and every live block's cached mean key (fp32)
-            r["select"] = roofline("qpool_kernel + score_mean_kernel", "hbm", B * n * row + B * P * H * D * 4, ms,
+            r["select"] = roofline("select_cached_kernel", "hbm", B * n * row + B * P * H * D * 4, ms,
                                    peaks, src)
             info = cache.info(0)
             sel = torch.empty((B, wl.n_top), dtype=torch.int32, device=dev)
@@ -455,9 +455,9 @@ def measure_block(pf, synth, dev, flush, stream, peaks, src, blocks=3) -> dict:
     cache.poll_device_error()
     r = {"ms_per_block": round(ms, 3), "layer_step_ms": round(ms / (L * S), 4), "context_tokens": Lk,
          "attention_flop_per_block": flops,
-         # attend per layer and step; qpool + score_mean per layer at step 0;
+         # attend per layer and step; the selection per layer at step 0;
          # copy + key mean per layer's append; one shift launch for all sinks
-         "launches_per_block": L * S + 2 * L + 2 * L + 1,
+         "launches_per_block": L * S + L + 2 * L + 1,
          "attend_block": roofline("attend_kernel (whole block: selection, appends and shifts included)", "tensor",
                                   flops, ms, peaks, src, sustained=True)}
     del cache, Qs, Ks, Vs, Kcs, O, blk
@@ -530,11 +530,11 @@ def run_gpu(args):
             dist.all_reduce(t, op=dist.ReduceOp.SUM)
 
     def select(q):
-        if sharded:
+        if sharded:   # scores on this rank's heads, then the top-k of the summed scores
             select_head_sharded(cache, 0, q, scores, H_all, all_reduce_sum, pf.ROUTE_SCORES_ONLY, pf.ROUTE_GIVEN)
-            return 3
-        cache.select_mid(0, q)
-        return 2
+            return 2
+        cache.select_mid(0, q)   # one launch
+        return 1
 
     def step(q, k, v, kc, vc, out, att_events=None):
         nl = select(q)
@@ -546,7 +546,7 @@ def run_gpu(args):
         ev = cache.append_block(0, k, v, kc, vc)
         if ev:
             cache.rope_shift(0, pf.PART_SINK, ev * wl.block_frames)
-        return LAUNCHES_PER_STEP_BASE - 2 + nl + (1 if ev else 0)
+        return LAUNCHES_PER_STEP_BASE + nl + (1 if ev else 0)
 
     clocks = ClockSampler(local)
     clocks.start()
