@@ -61,3 +61,31 @@ def test_peaks_come_from_the_measured_file_when_present():
         assert source == "measured"
     else:
         assert source == "fallback" and peaks
+
+
+def test_nvml_reason_bits_decode_to_the_rejecting_names():
+    # NVML's clock-event reason bits: sw power cap 0x4, hw slowdown 0x8,
+    # sw thermal 0x20, hw thermal 0x40, hw power brake 0x80; idle (0x1) and
+    # others are not reported
+    assert bench.reason_names(0) == []
+    assert bench.reason_names(0x1) == []
+    assert bench.reason_names(0x4) == ["sw_power_cap"]
+    assert bench.reason_names(0x8 | 0x40) == ["hw_slowdown", "hw_thermal_slowdown"]
+    assert bench.reason_names(0x20 | 0x80 | 0x1) == ["hw_power_brake_slowdown", "sw_thermal_slowdown"]
+
+
+def test_sampled_rows_summarised_inside_the_window():
+    rows = [(10.0, 1965.0, 1965.0, []), (10.5, 1900.0, 1965.0, ["sw_power_cap"]), (12.0, 800.0, 1965.0, ["hw_slowdown"])]
+    s = bench.summarize_rows(rows, 9.9, 11.0)
+    assert s == {"sm_mhz": 1932.5, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 2}
+    assert bench.summarize_rows(rows, 20.0, 30.0) is None
+
+
+def test_head_shards_and_roofline_record():
+    assert [bench.head_shard(12, 8, r) for r in range(8)] == [(0, 2), (2, 4), (4, 6), (6, 8), (8, 9), (9, 10),
+                                                             (10, 11), (11, 12)]
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    r = bench.roofline("k", "hbm", 6e9, 1.0, peaks, "measured")
+    assert r["achieved"] == 6000.0 and r["frac"] == 1.0 and r["unit"] == "GB/s"
+    r = bench.roofline("k", "tensor", 1.4e12, 1.0, peaks, "measured", sustained=True)
+    assert r["achieved"] == 1400.0 and r["frac"] == 1.0 and "sustained" in r["peak_source"]
