@@ -606,7 +606,7 @@ def test_generation_loop_against_oracle_model(pf, fused):
 
 def test_block_steps_across_layers_against_oracle_model(pf):
     """CFG batch 2 (cond + uncond), 2 layers, 4 denoising steps per block,
-    6 blocks.  pf_attend_step selects from the first step's queries and
+    8 blocks (two evictions).  pf_attend_step selects from the first step's queries and
     reuses that selection at steps 2-4 while the queries and the current
     block's K/V change from step to step; pf_finish_block appends the final
     block to every layer and shifts every sink on eviction.  The oracle keeps
@@ -618,7 +618,7 @@ def test_block_steps_across_layers_against_oracle_model(pf):
     cache = pf.PackedKVCache(pf.config_for(wl))
     model = [{"sinkK": [], "sinkV": [], "mid": [], "recent": []} for _ in range(L)]
     total_ev = 0
-    for i in range(6):
+    for i in range(8):
         final = [synth.make_block(wl, 7100 + 10 * i + l) for l in range(L)]
         for step in range(S):
             for l in range(L):
