@@ -139,7 +139,10 @@ Geometry geometry(const pf_config* c, bool* overflow) {
   const int slabs = g.HD / pf::kSelSlabCols;
   g.sel_bytes = z.bytes(B, c->n_top > 0 ? c->n_top : 1, 4);
   g.scores_bytes = z.bytes(B, g.slots, 4);
-  g.partial_bytes = z.bytes(B, g.slots, std::max(g.chunks_per_block, slabs), 4);
+  // slab-major partials with the slot stride padded to a multiple of 4
+  // (16-byte loads of four blocks' parts)
+  const size_t slots_pad = (static_cast<size_t>(g.slots) + 3) / 4 * 4;
+  g.partial_bytes = z.bytes(B, std::max(z.mul(g.slots, g.chunks_per_block), z.mul(slots_pad, slabs)), 4);
   g.qsum_bytes = z.bytes(B, pf::kSelMaxRowChunks, g.HD, 4);
   g.ticket_bytes = z.bytes(B, 1 + slabs, 4);
   g.kbar_bytes = z.bytes(B, g.slots, g.HD, 4);
@@ -617,10 +620,11 @@ pf_status pf_select_mid_ex(pf_cache* c, int layer, const void* Q, const pf_selec
   a.chunk_rows = g.chunk_rows;
   // one partial score per 64-column slab of the heads used, slab-major
   const int nslabs = (o.head_hi - o.head_lo) * pf::kHeadDim / pf::kSelSlabCols;
+  const int slots_pad = (g.slots + 3) / 4 * 4;
   a.chunks_per_block = nslabs;
   a.p_stride = 1;
-  a.k_stride = g.slots;
-  a.partial_ld = nslabs * g.slots;
+  a.k_stride = slots_pad;
+  a.partial_ld = nslabs * slots_pad;
   a.slab_ticket = Ly.ticket + cf.batch;
   {
     // row chunks per slab: about two CTAs per SM over the whole grid

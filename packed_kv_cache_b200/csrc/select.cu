@@ -144,20 +144,35 @@ __device__ unsigned block_exclusive_scan(unsigned v, unsigned* total) {
 // The last CTA of batch item b: block scores from the partial sums, exact
 // radix selection of the n_top largest (ties to the older block), outputs in
 // ascending age, and the cleanup that leaves ticket[b] zero.
+__device__ void select_topk_from_keys(const SelectArgs& a, int b, uint32_t* keys);
+
+// Block score q from its partial sums, in part order; stored as a sort key
+// and written out.
+__device__ __forceinline__ void put_score(const SelectArgs& a, int b, uint32_t* keys, int q, float s) {
+  s *= a.score_scale;
+  keys[q] = order_key(s);
+  a.scores[static_cast<long long>(b) * a.slots + q] = s;
+  if (a.scores_out) a.scores_out[static_cast<long long>(b) * a.count + q] = s;
+}
+
 __device__ void select_tail(const SelectArgs& a, int b, uint32_t* keys) {
-  __shared__ unsigned hist[256];
-  __shared__ unsigned sh_prefix, sh_need;
   const int t = threadIdx.x;
   const int count = a.count;
   for (int q = t; q < count; q += kThreads) {
     const float* pp = a.partial + static_cast<long long>(b) * a.partial_ld + static_cast<long long>(q) * a.p_stride;
     float s = 0.f;
     for (int k = 0; k < a.chunks_per_block; ++k) s += __ldcg(pp + static_cast<long long>(k) * a.k_stride);
-    s *= a.score_scale;
-    keys[q] = order_key(s);
-    a.scores[static_cast<long long>(b) * a.slots + q] = s;
-    if (a.scores_out) a.scores_out[static_cast<long long>(b) * count + q] = s;
+    put_score(a, b, keys, q, s);
   }
+  select_topk_from_keys(a, b, keys);
+}
+
+// keys[0 .. count) hold the block scores' sort keys (scores already written).
+__device__ void select_topk_from_keys(const SelectArgs& a, int b, uint32_t* keys) {
+  __shared__ unsigned hist[256];
+  __shared__ unsigned sh_prefix, sh_need;
+  const int t = threadIdx.x;
+  const int count = a.count;
   if (!a.topk) {   // scores only
     if (t == 0) a.ticket[b] = 0u;
     return;
@@ -396,8 +411,27 @@ __global__ void __launch_bounds__(kThreads, 3) select_cached_kernel(const Select
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  // ---- 3. scores (slab parts added in slab order) and the top-k
-  select_tail(a, b, keys);
+  // ---- 3. scores: the slab parts of four consecutive blocks per thread,
+  // added in slab order (16-byte loads, eight slabs in flight), then the top-k
+  {
+    const float* base = a.partial + static_cast<long long>(b) * a.partial_ld;
+    for (int q0 = 4 * t; q0 < a.count; q0 += 4 * kThreads) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+      for (int k = 0; k < nslabs; ++k) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(base + static_cast<long long>(k) * a.k_stride + q0));
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      const float r[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (q0 + e < a.count) put_score(a, b, keys, q0 + e, r[e]);
+    }
+  }
+  select_topk_from_keys(a, b, keys);
 }
 
 // kbar[b, slot] = mean over the block's n_c keys.  CTA (slot, b, z): 32
