@@ -383,9 +383,9 @@ def measure_stress(pf, synth, dev, flush, stream, peaks, src, iters) -> dict:
             rows = B * (wl.sink_blocks * n + P * nc + wl.recent_blocks * (n + nc))
             ms = timed_ms(lambda: cache.rope_shift(0, parts, 4), iters, flush, stream)
             # 22 rotary pairs = 88 bytes read and 88 written per (key, head)
-            r["rope_shift_all"] = roofline("rope_shift_tma_kernel", "hbm", rows * H * 176, ms, peaks, src)
+            r["rope_shift_all"] = roofline("rope_shift_kernel", "hbm", rows * H * 176, ms, peaks, src)
             ms = timed_ms(lambda: cache.rope_shift(0, pf.PART_SINK, 4), iters, flush, stream)
-            r["rope_shift_sink"] = roofline("rope_shift_tma_kernel", "hbm", B * wl.sink_blocks * n * H * 176, ms,
+            r["rope_shift_sink"] = roofline("rope_shift_kernel", "hbm", B * wl.sink_blocks * n * H * 176, ms,
                                             peaks, src)
         cache.select_mid(0, d["Q"])
         O = torch.empty_like(d["Q"])

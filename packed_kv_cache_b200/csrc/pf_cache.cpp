@@ -264,14 +264,11 @@ struct RunBuilder {
   pf::RopeTable tab;
   cudaStream_t st;
   bool f32 = false;  // runs of float32 vectors (cached mean keys) instead of bf16 keys
-  unsigned* dev_err = nullptr;
-  long long timeout_cycles = 0;
   cudaError_t err = cudaSuccess;
   RunBuilder() { runs.n = 0; runs.start[0] = 0; }
   void flush() {
     if (runs.n == 0) return;
-    cudaError_t e = f32 ? pf::launch_rope_shift_f32(runs, tab, st)
-                        : pf::launch_rope_shift(runs, tab, dev_err, timeout_cycles, st);
+    cudaError_t e = f32 ? pf::launch_rope_shift_f32(runs, tab, st) : pf::launch_rope_shift(runs, tab, st);
     if (e != cudaSuccess && err == cudaSuccess) err = e;
     runs.n = 0;
     runs.start[0] = 0;
@@ -695,8 +692,6 @@ pf_status pf_rope_shift(pf_cache* c, int layer, unsigned parts, int delta, void*
   const Geometry& g = c->g;
   RunBuilder rb, rm;
   rb.st = static_cast<cudaStream_t>(stream);
-  rb.dev_err = c->err;
-  rb.timeout_cycles = c->timeout_cycles;
   rm.st = rb.st;
   rm.f32 = true;
   rb.tab.pairs = cf.rope_split[0] / 2;

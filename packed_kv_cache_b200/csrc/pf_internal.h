@@ -113,10 +113,8 @@ __device__ __forceinline__ void rope_rotate_word(uint4& w, int word, const RopeT
 }
 #endif
 
-// bf16 key vectors, in place; a wait that gives up records a timeout in
-// *err (the cache's error word) after timeout_cycles SM clocks.
-cudaError_t launch_rope_shift(const RowRuns& runs, const RopeTable& tab, unsigned* err, long long timeout_cycles,
-                              cudaStream_t st);
+// bf16 key vectors, in place.
+cudaError_t launch_rope_shift(const RowRuns& runs, const RopeTable& tab, cudaStream_t st);
 // The same rotation of float32 128-dim vectors (cached mean keys); runs count vectors.
 cudaError_t launch_rope_shift_f32(const RowRuns& runs, const RopeTable& tab, cudaStream_t st);
 

@@ -434,37 +434,55 @@ __global__ void __launch_bounds__(kThreads, 3) select_cached_kernel(const Select
   select_topk_from_keys(a, b, keys);
 }
 
-// kbar[b, slot] = mean over the block's n_c keys.  CTA (slot, b, z): 32
-// column groups (16 bytes each) starting at group 32 z, rows split over the 8
-// warps; grid.x covers slots [slot0, slot0 + gridDim.x).
+// kbar[b, slot] = mean over the block's n_c keys.  CTA (slot, b, z): four
+// 16-byte column groups (32 dims) starting at group 4 z; thread t sums group
+// t % 4 over rows t / 4, t / 4 + 64, ... (all of a thread's rows in flight
+// for blocks of up to 256 rows), then a fixed-order reduction over the 64
+// row phases.  One appended block is HD / 32 CTAs (48 at 12 heads).
+constexpr int kMeanGroups = 4;
+constexpr int kMeanPhases = kThreads / kMeanGroups;
 __global__ void __launch_bounds__(kThreads) kmean_kernel(const void* pool_k, float* kbar, int slots, int n_c,
                                                          int HD, int slot0) {
-  __shared__ float red[kThreads / 32][32][9];
+  __shared__ float red[kThreads / 32][kMeanGroups][8];
   const int b = blockIdx.y;
   const int slot = slot0 + blockIdx.x;
   const int G = HD / 8;
-  const int lane = threadIdx.x & 31, phase = threadIdx.x >> 5;
-  const int g = blockIdx.z * 32 + lane;
-  const uint4* K = static_cast<const uint4*>(pool_k) + (static_cast<long long>(b) * slots + slot) * n_c * G;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int gl = t % kMeanGroups, phase = t / kMeanGroups;
+  const int g = blockIdx.z * kMeanGroups + gl;
+  const uint4* K = static_cast<const uint4*>(pool_k) + (static_cast<long long>(b) * slots + slot) * n_c * G + g;
   float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   if (g < G) {
-#pragma unroll 4
-    for (int r = phase; r < n_c; r += kThreads / 32) acc_bf16x8(acc, __ldg(K + static_cast<long long>(r) * G + g));
-  }
+    for (int r0 = phase; r0 < n_c; r0 += 4 * kMeanPhases) {
+      uint4 w[4];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) red[phase][lane][e] = acc[e];
-  __syncthreads();
-  if (phase == 0 && g < G) {
-    const float inv = 1.f / static_cast<float>(n_c);
+      for (int k = 0; k < 4; ++k) {
+        const int r = r0 + k * kMeanPhases;
+        w[k] = r < n_c ? __ldg(K + static_cast<long long>(r) * G) : make_uint4(0u, 0u, 0u, 0u);
+      }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      float s = 0.f;
-      for (int k = 0; k < kThreads / 32; ++k) s += red[k][lane][e];
-      acc[e] = s * inv;
+      for (int k = 0; k < 4; ++k) acc_bf16x8(acc, w[k]);
     }
-    float4* out = reinterpret_cast<float4*>(kbar + (static_cast<long long>(b) * slots + slot) * HD) + 2 * g;
-    out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  }
+  // lanes with the same group: l, l ^ 4, l ^ 8, ... (eight row phases per warp)
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 4);
+    acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 8);
+    acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+  }
+  if (lane < kMeanGroups) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[warp][lane][e] = acc[e];
+  }
+  __syncthreads();
+  if (t < kMeanGroups * 8) {
+    const int gg = t / 8, e = t % 8;
+    const int go = blockIdx.z * kMeanGroups + gg;
+    float sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) sum += red[w][gg][e];
+    if (go < G) kbar[(static_cast<long long>(b) * slots + slot) * HD + go * 8 + e] = sum / static_cast<float>(n_c);
   }
 }
 
@@ -539,7 +557,8 @@ cudaError_t launch_select_fifo(const SelectArgs& a, cudaStream_t st) {
 cudaError_t launch_kmean(const void* pool_k, float* kbar, int B, int slots, int n_c, int HD, int slot0, int nslots,
                          cudaStream_t st) {
   if (nslots <= 0) return cudaSuccess;
-  kmean_kernel<<<dim3(nslots, B, (HD / 8 + 31) / 32), kThreads, 0, st>>>(pool_k, kbar, slots, n_c, HD, slot0);
+  kmean_kernel<<<dim3(nslots, B, (HD / 8 + kMeanGroups - 1) / kMeanGroups), kThreads, 0, st>>>(pool_k, kbar, slots,
+                                                                                               n_c, HD, slot0);
   return cudaGetLastError();
 }
 

@@ -93,6 +93,9 @@ def test_static_selection_rejects_sizes_beyond_its_array(pf):
              dict(batch=1, heads=1, count=5000, n_c=4, slots=5000),
              dict(batch=1, heads=1, count=8, n_c=513, slots=8)]
     for c in cases:
+        # raw addresses: the library's own limits are under test, not the
+        # binding's size checks (nothing is launched: the sizes are refused first)
         with pytest.raises(pf.PFError) as e:
-            pf.pf_select_mid_static(Q, c["batch"], 64, c["heads"], K, c["slots"], c["n_c"], 0, c["count"], 4, sel)
+            pf.pf_select_mid_static(Q.data_ptr(), c["batch"], 64, c["heads"], K.data_ptr(), c["slots"], c["n_c"], 0,
+                                    c["count"], 4, sel.data_ptr())
         assert e.value.status_name == "PF_ERR_CAPACITY"
