@@ -139,11 +139,9 @@ Geometry geometry(const pf_config* c, bool* overflow) {
   const int slabs = g.HD / pf::kSelSlabCols;
   g.sel_bytes = z.bytes(B, c->n_top > 0 ? c->n_top : 1, 4);
   g.scores_bytes = z.bytes(B, g.slots, 4);
-  // slab-major partials with the slot stride padded to a multiple of 4
-  // (16-byte loads of four blocks' parts)
-  const size_t slots_pad = (static_cast<size_t>(g.slots) + 3) / 4 * 4;
-  g.partial_bytes = z.bytes(B, std::max(z.mul(g.slots, g.chunks_per_block), z.mul(slots_pad, slabs)), 4);
-  g.qsum_bytes = z.bytes(B, pf::kSelMaxRowChunks, g.HD, 4);
+  g.partial_bytes = z.bytes(B, g.slots, g.chunks_per_block, 4);
+  // per-row-chunk query sums, then their total
+  g.qsum_bytes = z.bytes(B, pf::kSelMaxRowChunks + 1, g.HD, 4);
   g.ticket_bytes = z.bytes(B, 1 + slabs, 4);
   g.kbar_bytes = z.bytes(B, g.slots, g.HD, 4);
   size_t t = z.mul(2, z.add(z.add(g.sink_bytes, g.pool_bytes), g.recent_bytes));
@@ -615,16 +613,18 @@ pf_status pf_select_mid_ex(pf_cache* c, int layer, const void* Q, const pf_selec
   a.head = Ly.mid_head;
   a.count = Ly.mid_count;
   a.chunk_rows = g.chunk_rows;
-  // one partial score per 64-column slab of the heads used, slab-major
+  // query sums over 64-column slabs of the heads used, in row chunks; then
+  // one dot product per block against its mean key
   const int nslabs = (o.head_hi - o.head_lo) * pf::kHeadDim / pf::kSelSlabCols;
-  const int slots_pad = (g.slots + 3) / 4 * 4;
-  a.chunks_per_block = nslabs;
+  a.qtot = Ly.qsum + static_cast<size_t>(cf.batch) * pf::kSelMaxRowChunks * g.HD;
+  a.chunks_per_block = 1;
   a.p_stride = 1;
-  a.k_stride = slots_pad;
-  a.partial_ld = nslabs * slots_pad;
+  a.k_stride = 1;
+  a.partial_ld = g.slots;
   a.slab_ticket = Ly.ticket + cf.batch;
   {
-    // row chunks per slab: about two CTAs per SM over the whole grid
+    // row chunks per slab: as many as keep the query-sum grid within one
+    // wave of two CTAs per SM
     static pf::PerDevice sm_count;
     int sms = 0;
     cudaError_t e = sm_count.get(&sms, [](int dev, int* v) {
@@ -632,7 +632,7 @@ pf_status pf_select_mid_ex(pf_cache* c, int layer, const void* Q, const pf_selec
     });
     if (e != cudaSuccess) return cuda_fail(e, "SM count");
     const long long per = 1LL * nslabs * cf.batch;
-    long long R = (2LL * sms + per - 1) / per;
+    long long R = (2LL * sms) / per;
     a.row_chunks = static_cast<int>(std::max(1LL, std::min<long long>(pf::kSelMaxRowChunks, R)));
   }
   const int rows = (g.n + o.q_stride - 1) / o.q_stride;

@@ -130,8 +130,8 @@ struct CopyRuns {
 cudaError_t launch_copy(const CopyRuns& runs, cudaStream_t st);
 
 // ------------------------------------------------------------- selection
-// The cache path's selection runs as one kernel over 64-column slabs of the
-// H * D query vector: kSelRowChunks chunks of query rows per slab at most.
+// The cache path's query sums run over 64-column slabs of the H * D query
+// vector, in at most kSelMaxRowChunks chunks of query rows per slab.
 constexpr int kSelSlabCols = 64;
 constexpr int kSelMaxRowChunks = 8;
 
@@ -140,6 +140,7 @@ struct SelectArgs {
   int B, n, HD;         // HD = H * D
   float* qsum;          // [B, HD] query sums (streaming path); [B, kSelMaxRowChunks, HD]
                         // per-row-chunk partial sums (cache path)
+  float* qtot;          // cache path: [B, HD] the chunks' sums added
   unsigned* slab_ticket;  // cache path: [B, HD / kSelSlabCols], zero on entry, left zero on exit
   int row_chunks;       // cache path: row chunks per slab (1 .. kSelMaxRowChunks)
   const void* pool_k;   // [B, slots, n_c, H, D] bf16
@@ -166,8 +167,8 @@ struct SelectArgs {
 
 // qpool + scoring of the streamed compressed keys (+ top-k unless a.topk == 0).
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
-// The same from the cached mean keys (a.kbar), as one kernel: query pooling
-// and the partial dot products per slab, then the top-k (unless a.topk == 0).
+// The same from the cached mean keys (a.kbar): query sums per slab, then one
+// dot product per block and the top-k (unless a.topk == 0), two kernels.
 cudaError_t launch_select_cached(const SelectArgs& a, cudaStream_t st);
 // Top-k of given scores: a.partial holds [B, partial_ld] scores by age
 // (chunks_per_block = 1, score_scale = 1).

@@ -10,15 +10,15 @@
 //   S[b, p] = qsum[b] . kbar[b, p] / (n H sqrt(D)),  kbar = the block's mean key,
 // so when the cache keeps each compressed block's mean key (computed once,
 // when the block enters the pool) scoring reads 6 KB per block instead of its
-// n_c keys.  That path is one kernel (select_cached_kernel): CTAs own a
-// 64-column slab of the H*D query vector and a chunk of the query rows; each
-// sums its rows' columns, the last row chunk of a slab (ticket) adds the
-// chunks and takes the slab's part of every block's dot product with its
-// mean key, and the last slab of a batch item (ticket) adds the slabs' parts
-// in a fixed order, runs an exact radix select of the n_top largest scores
-// (ties to the older block), writes the selection in ascending age, and
-// clears its tickets.  The allocation-free entry point has no cached means
-// and streams the keys with two kernels:
+// n_c keys.  That path is two kernels: qsum_slab_kernel sums the block's
+// queries (CTAs own a 64-column slab of the H*D query vector and a chunk of
+// its rows; the last chunk of a slab adds the chunks in a fixed order), and
+// score_cached_kernel, launched as a programmatic dependent so that it
+// fetches the mean keys while the sums are formed, takes one dot product per
+// block (a warp each) and, in the last CTA of a batch item (ticket), runs an
+// exact radix select of the n_top largest scores (ties to the older block),
+// writes the selection in ascending age, and clears its ticket.  The
+// allocation-free entry point has no cached means and streams the keys:
 //   1. qpool: the columns of Q[b] summed over the block's rows into qsum[b].
 //   2. score: one CTA per 32-row chunk of a pool block, a dot product with
 //      qsum[b]; the last CTA of batch item b (ticket counter) adds the chunks
@@ -303,135 +303,155 @@ __global__ void __launch_bounds__(kThreads, 5) score_kernel(const SelectArgs a) 
   select_tail(a, b, keys);
 }
 
-// The cache path's selection in one kernel.  CTA (x, b): slab x / R of the
-// score's column range [d_lo, d_hi) (kSelSlabCols columns), row chunk x % R
-// of the pooled query rows (R = a.row_chunks).
-//  1. column sums of the chunk's rows over the slab -> qsum[b, chunk, slab];
-//  2. the last chunk of the slab (slab ticket) adds the R chunk sums (in
-//     chunk order) and forms, for every live block, the slab's part of the
-//     dot product with the block's mean key -> partial[b, slab, age];
-//  3. the last slab (batch ticket) adds the parts (in slab order) and runs
-//     the top-k (select_tail).
-constexpr int kSelLoads = 8;   // row loads in flight per thread in step 1
-__global__ void __launch_bounds__(kThreads, 3) select_cached_kernel(const SelectArgs a) {
-  extern __shared__ float smem[];
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem);   // [count], the last CTA's top-k
+// The cache path's selection: two kernels, the second launched as a
+// programmatic dependent of the first so that it starts (and fetches the
+// mean keys, which do not depend on the first) while the first still runs.
+//
+// qsum_slab_kernel, CTA (x, b): slab x / R of the score's column range
+// [d_lo, d_hi) (kSelSlabCols columns), row chunk x % R of the pooled query
+// rows (R = a.row_chunks).  Column sums of the chunk's rows over the slab go
+// to qsum[b, chunk]; the chunk that finishes last (slab ticket) adds the R
+// chunk sums in chunk order into qtot[b] and clears the ticket.
+constexpr int kSelLoads = 16;   // row loads in flight per thread
+__global__ void __launch_bounds__(kThreads, 2) qsum_slab_kernel(const SelectArgs a) {
+  // let the scoring kernel be scheduled now: it waits for this grid's
+  // completion before reading qtot
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ float red[kThreads / 32][kSelSlabCols];
-  __shared__ float qs[kSelSlabCols];
   __shared__ unsigned is_last;
   const int b = blockIdx.y;
   const int R = a.row_chunks;
   const int slab = blockIdx.x / R, rc = blockIdx.x - slab * R;
-  const int nslabs = gridDim.x / R;
   const int col0 = a.d_lo + slab * kSelSlabCols;
   const int G = a.HD / 8;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  // ---- 1. column sums: thread t owns 16-byte group t % 8 of the slab in row phase t / 8
-  {
-    const int g = t & 7, phase = t >> 3;
-    constexpr int kPhases = kThreads / 8;
-    const int nr = (a.n + a.q_stride - 1) / a.q_stride;   // pooled rows 0, q_stride, 2 q_stride, ...
-    const int r_lo = static_cast<int>(static_cast<long long>(rc) * nr / R);
-    const int r_hi = static_cast<int>(static_cast<long long>(rc + 1) * nr / R);
-    const uint4* Q = static_cast<const uint4*>(a.Q) + static_cast<long long>(b) * a.n * G + col0 / 8 + g;
-    const long long row_step = static_cast<long long>(a.q_stride) * G;
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int r = r_lo + phase; r < r_hi; r += kSelLoads * kPhases) {
-      uint4 w[kSelLoads];
+  // thread t owns 16-byte group t % 8 of the slab in row phase t / 8: a warp
+  // reads four whole 128-byte row slices per load instruction
+  const int g = t & 7, phase = t >> 3;
+  constexpr int kPhases = kThreads / 8;
+  const int nr = (a.n + a.q_stride - 1) / a.q_stride;   // pooled rows 0, q_stride, 2 q_stride, ...
+  const int r_lo = static_cast<int>(static_cast<long long>(rc) * nr / R);
+  const int r_hi = static_cast<int>(static_cast<long long>(rc + 1) * nr / R);
+  const uint4* Q = static_cast<const uint4*>(a.Q) + static_cast<long long>(b) * a.n * G + col0 / 8 + g;
+  const long long row_step = static_cast<long long>(a.q_stride) * G;
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int r = r_lo + phase; r < r_hi; r += kSelLoads * kPhases) {
+    uint4 w[kSelLoads];
 #pragma unroll
-      for (int k = 0; k < kSelLoads; ++k) {
-        const int rr = r + k * kPhases;
-        w[k] = rr < r_hi ? __ldg(Q + rr * row_step) : make_uint4(0u, 0u, 0u, 0u);
-      }
+    for (int k = 0; k < kSelLoads; ++k) {
+      const int rr = r + k * kPhases;
+      w[k] = rr < r_hi ? __ldg(Q + rr * row_step) : make_uint4(0u, 0u, 0u, 0u);
+    }
 #pragma unroll
-      for (int k = 0; k < kSelLoads; ++k) acc_bf16x8(acc, w[k]);
-    }
-    // the four row phases of a warp hold the same group: lanes g, g + 8, g + 16, g + 24
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 8);
-      acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
-    }
-    if (lane < 8) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) red[warp][lane * 8 + e] = acc[e];
-    }
-    __syncthreads();
-    if (t < kSelSlabCols) {
-      float sum = 0.f;
-#pragma unroll
-      for (int w = 0; w < kThreads / 32; ++w) sum += red[w][t];
-      a.qsum[(static_cast<long long>(b) * kSelMaxRowChunks + rc) * a.HD + col0 + t] = sum;
-      __threadfence();
-    }
-    __syncthreads();
-    if (t == 0) {
-      __threadfence();
-      unsigned* tk = a.slab_ticket + static_cast<long long>(b) * (a.HD / kSelSlabCols) + slab;
-      is_last = (atomicAdd(tk, 1u) == static_cast<unsigned>(R - 1)) ? 1u : 0u;
-      if (is_last) *tk = 0u;   // every chunk of this slab has arrived: ready for the next launch
-    }
-    __syncthreads();
-    if (!is_last) return;
-    __threadfence();
+    for (int k = 0; k < kSelLoads; ++k) acc_bf16x8(acc, w[k]);
   }
-  // ---- 2. this slab's part of every live block's score
-  if (t < kSelSlabCols) {
-    float sum = 0.f;
-    for (int c = 0; c < R; ++c) sum += __ldcg(a.qsum + (static_cast<long long>(b) * kSelMaxRowChunks + c) * a.HD + col0 + t);
-    qs[t] = sum;
+  // the four row phases of a warp hold the same group: lanes g, g + 8, g + 16, g + 24
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 8);
+    acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+  }
+  if (lane < 8) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[warp][lane * 8 + e] = acc[e];
   }
   __syncthreads();
-  {
-    const float4* q4 = reinterpret_cast<const float4*>(qs);
-    float* part = a.partial + static_cast<long long>(b) * a.partial_ld + static_cast<long long>(slab) * a.k_stride;
-    // one block per thread per step: its 256 bytes (16 loads) in flight
-    for (int p = t; p < a.count; p += kThreads) {
-      int slot = a.head + p;
-      if (slot >= a.slots) slot -= a.slots;
-      const float4* k4 = reinterpret_cast<const float4*>(a.kbar + (static_cast<long long>(b) * a.slots + slot) * a.HD + col0);
-      float4 y[kSelSlabCols / 4];
+  if (t < kSelSlabCols) {
+    float sum = 0.f;
 #pragma unroll
-      for (int i = 0; i < kSelSlabCols / 4; ++i) y[i] = __ldg(k4 + i);
-      float acc = 0.f;
-#pragma unroll
-      for (int i = 0; i < kSelSlabCols / 4; ++i) {
-        const float4 x = q4[i];
-        acc = fmaf(x.x, y[i].x, fmaf(x.y, y[i].y, fmaf(x.z, y[i].z, fmaf(x.w, y[i].w, acc))));
-      }
-      part[p] = acc;
-    }
+    for (int w = 0; w < kThreads / 32; ++w) sum += red[w][t];
+    a.qsum[(static_cast<long long>(b) * kSelMaxRowChunks + rc) * a.HD + col0 + t] = sum;
+    __threadfence();
   }
-  __threadfence();
   __syncthreads();
   if (t == 0) {
     __threadfence();
-    is_last = (atomicAdd(&a.ticket[b], 1u) == static_cast<unsigned>(nslabs - 1)) ? 1u : 0u;
+    unsigned* tk = a.slab_ticket + static_cast<long long>(b) * (a.HD / kSelSlabCols) + slab;
+    is_last = (atomicAdd(tk, 1u) == static_cast<unsigned>(R - 1)) ? 1u : 0u;
+    if (is_last) *tk = 0u;   // every chunk of this slab has arrived: ready for the next launch
   }
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  // ---- 3. scores: the slab parts of four consecutive blocks per thread,
-  // added in slab order (16-byte loads, eight slabs in flight), then the top-k
-  {
-    const float* base = a.partial + static_cast<long long>(b) * a.partial_ld;
-    for (int q0 = 4 * t; q0 < a.count; q0 += 4 * kThreads) {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-      for (int k = 0; k < nslabs; ++k) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(base + static_cast<long long>(k) * a.k_stride + q0));
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
-      }
-      const float r[4] = {acc.x, acc.y, acc.z, acc.w};
+  if (t < kSelSlabCols) {
+    float sum = 0.f;
+    for (int c = 0; c < R; ++c) sum += __ldcg(a.qsum + (static_cast<long long>(b) * kSelMaxRowChunks + c) * a.HD + col0 + t);
+    a.qtot[static_cast<long long>(b) * a.HD + col0 + t] = sum;
+  }
+}
+
+// score_cached_kernel, CTA (x, b): warp w scores live block p = 8 x + w,
+// qtot[b] . kbar[b, slot(p)] over [d_lo, d_hi) (the whole mean key read by
+// the warp in 512-byte coalesced steps; the first kPreLoads steps issued
+// before waiting for qsum_slab_kernel); the last CTA of batch item b
+// (ticket) runs the top-k.
+constexpr int kPreLoads = 12;   // float4 loads per lane issued before the wait (all of them at 12 heads)
+__global__ void __launch_bounds__(kThreads, 2) score_cached_kernel(const SelectArgs a) {
+  extern __shared__ float smem[];
+  float* qs = smem;                                           // [HD] qtot[b] (only [d_lo, d_hi) is read)
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + a.HD);  // [count], the last CTA's top-k
+  __shared__ unsigned is_last;
+  const int b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int p = blockIdx.x * (kThreads / 32) + warp;
+  const int v_lo = a.d_lo / 4, v_hi = a.d_hi / 4;
+  const float4* k4 = nullptr;
+  float4 y[kPreLoads];
+  if (p < a.count) {
+    int slot = a.head + p;
+    if (slot >= a.slots) slot -= a.slots;
+    k4 = reinterpret_cast<const float4*>(a.kbar + (static_cast<long long>(b) * a.slots + slot) * a.HD);
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (q0 + e < a.count) put_score(a, b, keys, q0 + e, r[e]);
+    for (int u = 0; u < kPreLoads; ++u) {
+      const int i = v_lo + lane + 32 * u;
+      y[u] = i < v_hi ? __ldg(k4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
-  select_topk_from_keys(a, b, keys);
+  // the query sums of qsum_slab_kernel: complete and visible after this
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  for (int i = a.d_lo + threadIdx.x; i < a.d_hi; i += kThreads) qs[i] = __ldcg(a.qtot + static_cast<long long>(b) * a.HD + i);
+  __syncthreads();
+  if (p < a.count) {
+    const float4* q4 = reinterpret_cast<const float4*>(qs);
+    float acc = 0.f;
+#pragma unroll
+    for (int u = 0; u < kPreLoads; ++u) {
+      const int i = v_lo + lane + 32 * u;
+      if (i < v_hi) {
+        const float4 x = q4[i];
+        acc = fmaf(x.x, y[u].x, fmaf(x.y, y[u].y, fmaf(x.z, y[u].z, fmaf(x.w, y[u].w, acc))));
+      }
+    }
+    // more heads than the prefetch covers: the rest, eight loads in flight
+    for (int i0 = v_lo + lane + 32 * kPreLoads; i0 < v_hi; i0 += 32 * 8) {
+      float4 z[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + 32 * u;
+        z[u] = i < v_hi ? __ldg(k4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + 32 * u;
+        if (i < v_hi) {
+          const float4 x = q4[i];
+          acc = fmaf(x.x, z[u].x, fmaf(x.y, z[u].y, fmaf(x.z, z[u].z, fmaf(x.w, z[u].w, acc))));
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) a.partial[static_cast<long long>(b) * a.partial_ld + p] = acc;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    is_last = (atomicAdd(&a.ticket[b], 1u) == gridDim.x - 1u) ? 1u : 0u;
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  select_tail(a, b, keys);
 }
 
 // kbar[b, slot] = mean over the block's n_c keys.  CTA (slot, b, z): four
@@ -524,16 +544,29 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
 cudaError_t launch_select_cached(const SelectArgs& a, cudaStream_t st) {
   if (a.count <= 0) return cudaSuccess;
   const int nslabs = (a.d_hi - a.d_lo) / kSelSlabCols;
-  if (nslabs <= 0 || a.row_chunks < 1 || a.row_chunks > kSelMaxRowChunks || a.chunks_per_block != nslabs)
+  if (nslabs <= 0 || a.row_chunks < 1 || a.row_chunks > kSelMaxRowChunks || a.chunks_per_block != 1)
     return cudaErrorInvalidValue;
-  const size_t smem = static_cast<size_t>(a.count) * 4;
+  qsum_slab_kernel<<<dim3(nslabs * a.row_chunks, a.B), kThreads, 0, st>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = static_cast<size_t>(a.HD) * 4 + static_cast<size_t>(a.count) * 4;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(select_cached_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    e = cudaFuncSetAttribute(score_cached_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  select_cached_kernel<<<dim3(nslabs * a.row_chunks, a.B), kThreads, smem, st>>>(a);
-  return cudaGetLastError();
+  // a programmatic dependent launch: scheduled while qsum_slab_kernel runs,
+  // it waits (griddepcontrol.wait) for that grid before reading its sums
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((a.count + kThreads / 32 - 1) / (kThreads / 32), a.B);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, score_cached_kernel, a);
 }
 
 cudaError_t launch_topk_given(const SelectArgs& a, cudaStream_t st) {
@@ -682,6 +715,7 @@ extern "C" pf_status pf_select_mid_static(const void* Q, int batch, int n, int h
   a.p_stride = a.chunks_per_block;
   a.k_stride = 1;
   a.slab_ticket = nullptr;
+  a.qtot = nullptr;
   a.row_chunks = 1;
   e = launch_select(a, st);
   if (e != cudaSuccess)
