@@ -369,7 +369,7 @@ def measure_stress(pf, synth, dev, flush, stream, peaks, src, iters) -> dict:
         if name == "stress16":
             ms = timed_ms(lambda: cache.select_mid(0, d["Q"]), iters, flush, stream)
             # reads: the queries (bf16) and every live block's cached mean key (fp32)
-            r["select"] = roofline("select_cached_kernel", "hbm", B * n * row + B * P * H * D * 4, ms,
+            r["select"] = roofline("qsum_slab_kernel + score_cached_kernel", "hbm", B * n * row + B * P * H * D * 4, ms,
                                    peaks, src)
             info = cache.info(0)
             sel = torch.empty((B, wl.n_top), dtype=torch.int32, device=dev)
