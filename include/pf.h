@@ -188,7 +188,9 @@ pf_status pf_cache_load_mid(pf_cache* cache, int layer, const void* Kc, const vo
  * sel_out (optional, device, [B, min(n_top, mid_count)] int32): the chosen
  * blocks by age (0 = oldest live block), ascending.
  * scores_out (optional, device, [B, mid_count] float): S by age.
- * One kernel launch; no host synchronisation.
+ * Two kernel launches (the query sums, then the scores and the top-k as a
+ * programmatic dependent launch that starts while the sums are formed); no
+ * host synchronisation.
  */
 pf_status pf_select_mid(pf_cache* cache, int layer, const void* Q, int32_t* sel_out,
                         float* scores_out, void* stream);
@@ -232,8 +234,9 @@ typedef struct pf_select_opts {
  * pf_select_mid with a routing policy (see above).  opts NULL = the method's
  * defaults (PF_ROUTE_SCORE, every query row, every head) = pf_select_mid.
  * sel_out / scores_out as for pf_select_mid (scores_out is required for
- * PF_ROUTE_SCORES_ONLY and ignored by PF_ROUTE_FIFO).  Every policy
- * launches one kernel.  Errors: PF_ERR_ARG for a bad policy, stride, head range, or a
+ * PF_ROUTE_SCORES_ONLY and ignored by PF_ROUTE_FIFO).  PF_ROUTE_SCORE and
+ * PF_ROUTE_SCORES_ONLY launch two kernels, PF_ROUTE_GIVEN and PF_ROUTE_FIFO
+ * one.  Errors: PF_ERR_ARG for a bad policy, stride, head range, or a
  * missing scores_in / scores_out.
  */
 pf_status pf_select_mid_ex(pf_cache* cache, int layer, const void* Q, const pf_select_opts* opts,
@@ -285,8 +288,8 @@ pf_status pf_attend(pf_cache* cache, int layer, const void* Q, const void* K_cur
  * step's queries, then pf_attend; step > 0: pf_attend with the selection
  * stored at step 0 (PF_ERR_STATE if the pool changed since, or if no
  * selection was made while the pool holds more than n_top blocks).
- * Arguments as for pf_attend; step >= 0.  Two or three kernel launches at
- * step 0, one after.
+ * Arguments as for pf_attend; step >= 0.  Three kernel launches at step 0
+ * (selection, attention), one after.
  */
 pf_status pf_attend_step(pf_cache* cache, int layer, int step, const void* Q, const void* K_cur,
                          const void* V_cur, void* O, float* lse, void* stream);
