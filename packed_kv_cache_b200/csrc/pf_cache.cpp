@@ -615,7 +615,8 @@ pf_status pf_select_mid_ex(pf_cache* c, int layer, const void* Q, const pf_selec
   a.chunk_rows = g.chunk_rows;
   // query sums over 64-column slabs of the heads used, in row chunks; then
   // one dot product per block against its mean key
-  const int nslabs = (o.head_hi - o.head_lo) * pf::kHeadDim / pf::kSelSlabCols;
+  const int nslabs = (o.head_hi - o.head_lo) * pf::kHeadDim /
+                     pf::select_slab_cols(o.head_lo * pf::kHeadDim, o.head_hi * pf::kHeadDim);
   a.qtot = Ly.qsum + static_cast<size_t>(cf.batch) * pf::kSelMaxRowChunks * g.HD;
   a.chunks_per_block = 1;
   a.p_stride = 1;

@@ -130,10 +130,13 @@ struct CopyRuns {
 cudaError_t launch_copy(const CopyRuns& runs, cudaStream_t st);
 
 // ------------------------------------------------------------- selection
-// The cache path's query sums run over 64-column slabs of the H * D query
-// vector, in at most kSelMaxRowChunks chunks of query rows per slab.
-constexpr int kSelSlabCols = 64;
-constexpr int kSelMaxRowChunks = 8;
+// The cache path's query sums run over slabs of 256 columns of the H * D
+// query vector (128 when the score's column range is an odd number of
+// heads), in at most kSelMaxRowChunks chunks of query rows per slab.
+// kSelSlabCols is the narrowest slab (it sizes the slab tickets).
+constexpr int kSelSlabCols = 128;
+constexpr int kSelMaxRowChunks = 32;
+inline int select_slab_cols(int d_lo, int d_hi) { return ((d_hi - d_lo) % 256 == 0) ? 256 : 128; }
 
 struct SelectArgs {
   const void* Q;        // [B, n, H, D] bf16

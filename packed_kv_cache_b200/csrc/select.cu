@@ -308,27 +308,31 @@ __global__ void __launch_bounds__(kThreads, 5) score_kernel(const SelectArgs a) 
 // mean keys, which do not depend on the first) while the first still runs.
 //
 // qsum_slab_kernel, CTA (x, b): slab x / R of the score's column range
-// [d_lo, d_hi) (kSelSlabCols columns), row chunk x % R of the pooled query
-// rows (R = a.row_chunks).  Column sums of the chunk's rows over the slab go
-// to qsum[b, chunk]; the chunk that finishes last (slab ticket) adds the R
-// chunk sums in chunk order into qtot[b] and clears the ticket.
+// [d_lo, d_hi) (kGroups * 8 columns: 256, or 128 when the range is an odd
+// number of heads), row chunk x % R of the pooled query rows (R =
+// a.row_chunks).  A warp reads 32 / kGroups whole rows of the slab per load
+// instruction (512 contiguous bytes of a row at 256 columns).  Column sums of
+// the chunk's rows go to qsum[b, chunk]; the chunk that finishes last (slab
+// ticket) adds the R chunk sums in chunk order into qtot[b] and clears the
+// ticket.
 constexpr int kSelLoads = 16;   // row loads in flight per thread
+template <int kGroups>
 __global__ void __launch_bounds__(kThreads, 2) qsum_slab_kernel(const SelectArgs a) {
   // let the scoring kernel be scheduled now: it waits for this grid's
   // completion before reading qtot
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  __shared__ float red[kThreads / 32][kSelSlabCols];
+  constexpr int kCols = kGroups * 8;
+  constexpr int kPhases = kThreads / kGroups;
+  __shared__ float red[kThreads / 32][kCols];
   __shared__ unsigned is_last;
   const int b = blockIdx.y;
   const int R = a.row_chunks;
   const int slab = blockIdx.x / R, rc = blockIdx.x - slab * R;
-  const int col0 = a.d_lo + slab * kSelSlabCols;
+  const int col0 = a.d_lo + slab * kCols;
   const int G = a.HD / 8;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  // thread t owns 16-byte group t % 8 of the slab in row phase t / 8: a warp
-  // reads four whole 128-byte row slices per load instruction
-  const int g = t & 7, phase = t >> 3;
-  constexpr int kPhases = kThreads / 8;
+  // thread t owns 16-byte group t % kGroups of the slab in row phase t / kGroups
+  const int g = t % kGroups, phase = t / kGroups;
   const int nr = (a.n + a.q_stride - 1) / a.q_stride;   // pooled rows 0, q_stride, 2 q_stride, ...
   const int r_lo = static_cast<int>(static_cast<long long>(rc) * nr / R);
   const int r_hi = static_cast<int>(static_cast<long long>(rc + 1) * nr / R);
@@ -345,18 +349,18 @@ __global__ void __launch_bounds__(kThreads, 2) qsum_slab_kernel(const SelectArgs
 #pragma unroll
     for (int k = 0; k < kSelLoads; ++k) acc_bf16x8(acc, w[k]);
   }
-  // the four row phases of a warp hold the same group: lanes g, g + 8, g + 16, g + 24
+  // lanes of a warp with the same group (32 / kGroups row phases)
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 8);
-    acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+  for (int off = kGroups; off < 32; off <<= 1) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
   }
-  if (lane < 8) {
+  if (lane < kGroups) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) red[warp][lane * 8 + e] = acc[e];
   }
   __syncthreads();
-  if (t < kSelSlabCols) {
+  if (t < kCols) {
     float sum = 0.f;
 #pragma unroll
     for (int w = 0; w < kThreads / 32; ++w) sum += red[w][t];
@@ -373,9 +377,17 @@ __global__ void __launch_bounds__(kThreads, 2) qsum_slab_kernel(const SelectArgs
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  if (t < kSelSlabCols) {
+  if (t < kCols) {
+    // the R chunk sums in chunk order, eight loads in flight
+    const float* src = a.qsum + static_cast<long long>(b) * kSelMaxRowChunks * a.HD + col0 + t;
     float sum = 0.f;
-    for (int c = 0; c < R; ++c) sum += __ldcg(a.qsum + (static_cast<long long>(b) * kSelMaxRowChunks + c) * a.HD + col0 + t);
+    for (int c0 = 0; c0 < R; c0 += 8) {
+      float v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[k] = c0 + k < R ? __ldcg(src + static_cast<long long>(c0 + k) * a.HD) : 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sum += v[k];
+    }
     a.qtot[static_cast<long long>(b) * a.HD + col0 + t] = sum;
   }
 }
@@ -543,10 +555,15 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
 
 cudaError_t launch_select_cached(const SelectArgs& a, cudaStream_t st) {
   if (a.count <= 0) return cudaSuccess;
-  const int nslabs = (a.d_hi - a.d_lo) / kSelSlabCols;
+  const int cols = a.d_hi - a.d_lo;
+  const int slab_cols = select_slab_cols(a.d_lo, a.d_hi);
+  const int nslabs = cols / slab_cols;
   if (nslabs <= 0 || a.row_chunks < 1 || a.row_chunks > kSelMaxRowChunks || a.chunks_per_block != 1)
     return cudaErrorInvalidValue;
-  qsum_slab_kernel<<<dim3(nslabs * a.row_chunks, a.B), kThreads, 0, st>>>(a);
+  if (slab_cols == 256)
+    qsum_slab_kernel<32><<<dim3(nslabs * a.row_chunks, a.B), kThreads, 0, st>>>(a);
+  else
+    qsum_slab_kernel<16><<<dim3(nslabs * a.row_chunks, a.B), kThreads, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t smem = static_cast<size_t>(a.HD) * 4 + static_cast<size_t>(a.count) * 4;

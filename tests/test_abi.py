@@ -60,10 +60,10 @@ def test_cache_bytes_layout(pf):
     al = lambda x: (x + 255) // 256 * 256  # noqa: E731
     slots = wl.mid_capacity + wl.recent_blocks
     cpb = (182 + 31) // 32
-    slabs = 12 * 128 // 64                  # the selection's 64-column slabs of the H * D vector
+    slabs = 12 * 128 // 128                 # slab tickets: one per 128 columns of the H * D vector
     per_layer = (2 * (al(2 * 6240 * row) + al(slots * 182 * row) + al(6240 * row))
                  + al(16 * 4) + al(slots * 4) + al(slots * cpb * 4)
-                 + al(9 * 12 * 128 * 4)     # query sums of up to 8 row chunks, then their total
+                 + al(33 * 12 * 128 * 4)    # query sums of up to 32 row chunks, then their total
                  + al((1 + slabs) * 4)      # batch and slab tickets
                  + al(slots * 1536 * 4))    # mean key of every pool slot
     # shared attention scratch: 256 split-tail slots of 128x128 fp32 partial
