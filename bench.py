@@ -455,9 +455,9 @@ def measure_block(pf, synth, dev, flush, stream, peaks, src, blocks=3) -> dict:
     cache.poll_device_error()
     r = {"ms_per_block": round(ms, 3), "layer_step_ms": round(ms / (L * S), 4), "context_tokens": Lk,
          "attention_flop_per_block": flops,
-         # attend per layer and step; the selection per layer at step 0;
-         # copy + key mean per layer's append; one shift launch for all sinks
-         "launches_per_block": L * S + L + 2 * L + 1,
+         # attend per layer and step; the selection's two kernels per layer at
+         # step 0; copy + key mean per layer's append; one shift launch for all sinks
+         "launches_per_block": L * S + 2 * L + 2 * L + 1,
          "attend_block": roofline("attend_kernel (whole block: selection, appends and shifts included)", "tensor",
                                   flops, ms, peaks, src, sustained=True)}
     del cache, Qs, Ks, Vs, Kcs, O, blk
@@ -530,11 +530,11 @@ def run_gpu(args):
             dist.all_reduce(t, op=dist.ReduceOp.SUM)
 
     def select(q):
-        if sharded:   # scores on this rank's heads, then the top-k of the summed scores
+        if sharded:   # scores on this rank's heads (2 launches), then the top-k of the summed scores (1)
             select_head_sharded(cache, 0, q, scores, H_all, all_reduce_sum, pf.ROUTE_SCORES_ONLY, pf.ROUTE_GIVEN)
-            return 2
-        cache.select_mid(0, q)   # one launch
-        return 1
+            return 3
+        cache.select_mid(0, q)   # query sums, then scores and top-k
+        return 2
 
     def step(q, k, v, kc, vc, out, att_events=None):
         nl = select(q)
