@@ -378,14 +378,16 @@ __global__ void __launch_bounds__(kThreads, 2) qsum_slab_kernel(const SelectArgs
   if (!is_last) return;
   __threadfence();
   if (t < kCols) {
-    // the R chunk sums in chunk order, all of them in flight at once
+    // the R chunk sums in chunk order, eight loads in flight
     const float* src = a.qsum + static_cast<long long>(b) * kSelMaxRowChunks * a.HD + col0 + t;
-    float v[kSelMaxRowChunks];
-#pragma unroll
-    for (int k = 0; k < kSelMaxRowChunks; ++k) v[k] = k < R ? __ldcg(src + static_cast<long long>(k) * a.HD) : 0.f;
     float sum = 0.f;
+    for (int c0 = 0; c0 < R; c0 += 8) {
+      float v[8];
 #pragma unroll
-    for (int k = 0; k < kSelMaxRowChunks; ++k) sum += v[k];
+      for (int k = 0; k < 8; ++k) v[k] = c0 + k < R ? __ldcg(src + static_cast<long long>(c0 + k) * a.HD) : 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sum += v[k];
+    }
     a.qtot[static_cast<long long>(b) * a.HD + col0 + t] = sum;
   }
 }
