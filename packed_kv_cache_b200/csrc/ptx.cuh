@@ -44,19 +44,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking check that the phase of `bar` with the given parity completed.
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Wait for the phase of `bar` with the given parity to complete.  Gives up
 // when *abort becomes non-zero or after `limit` SM clock cycles; on a
 // timeout it sets *abort and records `code` in *err.  Returns true if the
@@ -202,15 +189,6 @@ __device__ __forceinline__ void tmem_ld128_wait(uint32_t taddr, uint32_t* r) {
                : "r"(taddr), "r"(taddr + 32u), "r"(taddr + 64u), "r"(taddr + 96u) : "memory");
 }
 
-// 64 consecutive TMEM columns (two 32-column loads), then one wait.
-__device__ __forceinline__ void tmem_ld64_wait(uint32_t taddr, uint32_t* r) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%64];\n\t"
-               "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%65];\n\t"
-               "tcgen05.wait::ld.sync.aligned;"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
-               : "r"(taddr), "r"(taddr + 32u) : "memory");
-}
-
 // store 16 consecutive TMEM columns of this thread's lane (no wait).
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
@@ -229,22 +207,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 2^x on the FMA and integer pipes: x = n + f, n = round(x) (by adding and
-// subtracting 1.5 * 2^23), f in [-1/2, 1/2]; 2^f by a cubic fitted for the
-// least maximum relative error (7.5e-5; the fit is tests/fit_exp2.py);
-// 2^n added to the exponent bits.  x is clamped below at -126, so the
-// smallest result is about 1.2e-38 instead of 0 (at the clamp the cubic is
-// just under 1 and the sum falls into the subnormal encoding: 1.17533e-38).
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  float p = fmaf(5.517166906e-02f, f, 2.426111222e-01f);
-  p = fmaf(p, f, 6.932609855e-01f);
-  p = fmaf(p, f, 9.999280735e-01f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 // max of three floats (one instruction)
@@ -269,28 +231,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
-}
-
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
-// ex2_poly on both lanes of a pair: the rounding, the reduction and the
-// cubic as paired fp32 instructions, the exponent insertion as one
-// shift-and-add per lane.
-__device__ __forceinline__ uint64_t ex2_poly_x2(uint64_t x) {
-  x = f2_pack(fmaxf(f2_lo(x), -126.0f), fmaxf(f2_hi(x), -126.0f));
-  const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
-  const uint64_t t = f2_add(x, magic);
-  const uint64_t f = f2_sub(x, f2_sub(t, magic));
-  uint64_t p = f2_fma(f2_pack(5.517166906e-02f, 5.517166906e-02f), f, f2_pack(2.426111222e-01f, 2.426111222e-01f));
-  p = f2_fma(p, f, f2_pack(6.932609855e-01f, 6.932609855e-01f));
-  p = f2_fma(p, f, f2_pack(9.999280735e-01f, 9.999280735e-01f));
-  const uint32_t lo = static_cast<uint32_t>(p) + (static_cast<uint32_t>(t) << 23);
-  const uint32_t hi = static_cast<uint32_t>(p >> 32) + (static_cast<uint32_t>(t >> 32) << 23);
-  return (static_cast<uint64_t>(hi) << 32) | lo;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
