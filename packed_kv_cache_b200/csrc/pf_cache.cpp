@@ -613,8 +613,9 @@ pf_status pf_select_mid_ex(pf_cache* c, int layer, const void* Q, const pf_selec
   a.head = Ly.mid_head;
   a.count = Ly.mid_count;
   a.chunk_rows = g.chunk_rows;
-  // query sums over 64-column slabs of the heads used, in row chunks; then
-  // one dot product per block against its mean key
+  // query sums over 256-column slabs (128 for an odd head count) of the
+  // heads used, in row chunks; then one dot product per block against its
+  // mean key
   const int nslabs = (o.head_hi - o.head_lo) * pf::kHeadDim /
                      pf::select_slab_cols(o.head_lo * pf::kHeadDim, o.head_hi * pf::kHeadDim);
   a.qtot = Ly.qsum + static_cast<size_t>(cf.batch) * pf::kSelMaxRowChunks * g.HD;

@@ -11,7 +11,7 @@
 // so when the cache keeps each compressed block's mean key (computed once,
 // when the block enters the pool) scoring reads 6 KB per block instead of its
 // n_c keys.  That path is two kernels: qsum_slab_kernel sums the block's
-// queries (CTAs own a 64-column slab of the H*D query vector and a chunk of
+// queries (CTAs own a 256-column slab of the H*D query vector and a chunk of
 // its rows; the last chunk of a slab adds the chunks in a fixed order), and
 // score_cached_kernel, launched as a programmatic dependent so that it
 // fetches the mean keys while the sums are formed, takes one dot product per
@@ -642,7 +642,6 @@ struct StaticSelectScratch {
 
 static __device__ __align__(256) unsigned char g_select_scratch[sizeof(StaticSelectScratch)];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxDevices] = {};
 
