@@ -703,6 +703,37 @@ def test_block_step_calls_refuse_bad_arguments(pf):
     assert cache.info(1)["blocks_seen"] == wl.sink_blocks
 
 
+def test_later_steps_refuse_a_selection_the_pool_has_outgrown(pf):
+    # the selection made at a block's first step belongs to that pool: once
+    # the block is finished (the pool changed), a later-step call without a
+    # new first step is refused, and a first step selects again
+    L = 2
+    wl = _wl("ragged_a").replace(mid_capacity=3, n_top=2, planted=0, layers=L)
+    B, n, H, D = wl.batch, wl.n, wl.heads, wl.head_dim
+    cache = pf.PackedKVCache(pf.config_for(wl))
+    for i in range(7):
+        blks = [synth.make_block(wl, 800 + 10 * i + l) for l in range(L)]
+        cache.finish_block([b_["K"].cuda() for b_ in blks], [b_["V"].cuda() for b_ in blks],
+                           [b_["Kc"].cuda() for b_ in blks], [b_["Vc"].cuda() for b_ in blks])
+    assert cache.info(0)["mid_count"] == 3 > wl.n_top
+    Q = synth.bf16_normal((B, n, H, D), 900).cuda()
+    K = synth.bf16_normal((B, n, H, D), 901).cuda()
+    for l in range(L):
+        cache.attend_step(l, 0, Q, K, K)
+        cache.attend_step(l, 3, Q, K, K)                 # the stored selection is reused
+    blks = [synth.make_block(wl, 990 + l) for l in range(L)]
+    cache.finish_block([b_["K"].cuda() for b_ in blks], [b_["V"].cuda() for b_ in blks],
+                       [b_["Kc"].cuda() for b_ in blks], [b_["Vc"].cuda() for b_ in blks])
+    for l in range(L):
+        assert cache.info(l)["selection_valid"] == 0
+        with pytest.raises(pf.PFError) as e:
+            cache.attend_step(l, 1, Q, K, K)
+        assert e.value.status_name == "PF_ERR_STATE"
+        cache.attend_step(l, 0, Q, K, K)
+        assert cache.info(l)["selection_valid"] == 1
+    assert cache.poll_device_error() == 0
+
+
 @pytest.mark.parametrize("name", ["ragged_a", "ragged_c", "layer"])
 def test_sink_rope_in_attention_matches_oracle(pf, name):
     # the sink's shift recorded by pf_rope_shift and applied by pf_attend to
