@@ -64,6 +64,8 @@ constexpr uint32_t kOffV = kOffK + kKStages * kTileBytes;       // kVStages tile
 constexpr uint32_t kOffBar = kOffV + kVStages * kTileBytes;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;           // + barriers + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory");
+// the MMA issuer offsets operand descriptors in their 14-bit address field
+static_assert(kSmemBytes + 1024 < (1u << 18), "shared addresses fit a descriptor's address field");
 
 struct Bars {
   uint64_t q_full;
@@ -354,66 +356,72 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
       // ---------------------------------------------------------- MMA issuer
       const uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, 0);
       const uint32_t idesc_pv = idesc_bf16_f32(kBM, kHeadDim, 1);
-      const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
-      const uint32_t tO[2] = {tmem + 256u, tmem + 384u};
+      // Every operand descriptor is the tile's base descriptor plus a
+      // constant: the start-address field (bits 0-13) holds address / 16 and
+      // shared addresses stay below 2^18 bytes, so adding an offset / 16
+      // never carries out of the field.
+      const uint64_t dq = sdesc_sw128(sQ, 16, 1024);
+      const uint64_t dk = sdesc_sw128(sK, 16, 1024);
+      const uint64_t dv = sdesc_sw128(sV, kHalfBytes, 1024);
+      const int j0 = un.j0, j1 = un.j1, nqt = nq;
       auto issue_qk = [&](int t, int st) {
-        const uint32_t qa = sQ + t * kTileBytes, ka = sK + st * kTileBytes;
+        const uint64_t qa = dq + static_cast<uint32_t>(t) * (kTileBytes >> 4);
+        const uint64_t ka = dk + static_cast<uint32_t>(st) * (kTileBytes >> 4);
+        const uint32_t d = tmem + static_cast<uint32_t>(t) * 128u;
 #pragma unroll
         for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          mma_ss(tS[t], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idesc_qk, kk > 0);
+          const uint32_t off = (((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
+          mma_ss(d, qa + off, ka + off, idesc_qk, kk > 0);
         }
       };
       auto issue_pv = [&](int t, int st, bool first) {
-        const uint32_t va = sV + st * kTileBytes;
+        const uint64_t va = dv + static_cast<uint32_t>(st) * (kTileBytes >> 4);
+        const uint32_t d = tmem + 256u + static_cast<uint32_t>(t) * 128u;
+        const uint32_t a = tmem + static_cast<uint32_t>(t) * 128u;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ts(tO[t], tS[t] + kk * 8, sdesc_sw128(va + kk * 2048, kHalfBytes, 1024), idesc_pv,
-                 (!first || kk > 0) ? 1u : 0u);
+          mma_ts(d, a + kk * 8, va + kk * (2048 >> 4), idesc_pv, (!first || kk > 0) ? 1u : 0u);
       };
       uint64_t* k_avail = p.rotate_sink ? bars.k_ready : bars.k_full;
-      auto wait_k = [&](int g, unsigned site) {
-        return mbar_wait_bounded(&k_avail[g % kKStages], (g / kKStages) & 1, abort_flag, p.err,
-                                 kDevErrTimeoutBase | site, lim);
-      };
-      int kg = 0, vg = 0;
+      // ring positions kept as slot + phase
+      int ks = 0, vs = 0;
+      uint32_t kph = 0, vph = 0;
       bool ok = mbar_wait_bounded(&bars.q_full, 0, abort_flag, p.err, kDevErrTimeoutBase | 4u, lim);
-      if (ok) ok = wait_k(kg, 5u);
+      if (ok) ok = mbar_wait_bounded(&k_avail[ks], kph, abort_flag, p.err, kDevErrTimeoutBase | 5u, lim);
       if (ok) {
         tc_fence_after();
-        for (int t = 0; t < nq; ++t) {
-          issue_qk(t, kg % kKStages);
+        for (int t = 0; t < nqt; ++t) {
+          issue_qk(t, ks);
           mma_commit(&bars.s_full[t]);
         }
-        mma_commit(&bars.k_empty[kg % kKStages]);
-        ++kg;
+        mma_commit(&bars.k_empty[ks]);
+        if (++ks == kKStages) { ks = 0; kph ^= 1u; }
       }
-      for (int j = un.j0; ok && j < un.j1; ++j) {
-        const bool more = j + 1 < un.j1;
-        const int vs = vg % kVStages;
-        ok = mbar_wait_bounded(&bars.v_full[vs], (vg / kVStages) & 1, abort_flag, p.err, kDevErrTimeoutBase | 6u,
-                               lim);
-        for (int t = 0; ok && t < nq; ++t) {
-          ok = mbar_wait_bounded(&bars.p_full[t], (j - un.j0) & 1, abort_flag, p.err, kDevErrTimeoutBase | 7u, lim);
+      for (int j = j0; ok && j < j1; ++j) {
+        const bool more = j + 1 < j1;
+        const uint32_t pph = static_cast<uint32_t>(j - j0) & 1u;
+        ok = mbar_wait_bounded(&bars.v_full[vs], vph, abort_flag, p.err, kDevErrTimeoutBase | 6u, lim);
+        for (int t = 0; ok && t < nqt; ++t) {
+          ok = mbar_wait_bounded(&bars.p_full[t], pph, abort_flag, p.err, kDevErrTimeoutBase | 7u, lim);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(t, vs, j == un.j0);
+          issue_pv(t, vs, j == j0);
           if (more) {
             // S_t of the next tile overwrites P_t (tcgen05 MMAs issued by
             // one thread run in issue order: P_t V has read P_t by then)
-            if (t == 0) ok = wait_k(kg, 10u);
+            if (t == 0) ok = mbar_wait_bounded(&k_avail[ks], kph, abort_flag, p.err, kDevErrTimeoutBase | 10u, lim);
             if (!ok) break;
             tc_fence_after();
-            issue_qk(t, kg % kKStages);
+            issue_qk(t, ks);
             mma_commit(&bars.s_full[t]);
           }
         }
         if (!ok) break;
         mma_commit(&bars.v_empty[vs]);
-        ++vg;
+        if (++vs == kVStages) { vs = 0; vph ^= 1u; }
         if (more) {
-          mma_commit(&bars.k_empty[kg % kKStages]);
-          ++kg;
+          mma_commit(&bars.k_empty[ks]);
+          if (++ks == kKStages) { ks = 0; kph ^= 1u; }
         }
       }
       for (int t = 0; t < nq; ++t) mma_commit(&bars.o_final[t]);
