@@ -75,7 +75,6 @@ struct Bars {
   uint64_t s_full[2], p_full[2], o_final[2];
   uint32_t tmem_base;
   int abort;
-  int merge;
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
 
@@ -229,10 +228,6 @@ __device__ __forceinline__ void exp_chunk(const uint32_t* c, uint32_t dst, uint6
   tmem_st16(dst, pk);
 }
 
-__device__ __forceinline__ void named_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 __device__ __forceinline__ void store_row_bf16(uint4* dst, const float* o, float inv) {
 #pragma unroll
   for (int v = 0; v < 4; ++v) {
@@ -277,7 +272,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
       mbar_init(&bars.o_final[t], 1);
     }
     bars.abort = 0;
-    bars.merge = 0;
     fence_mbar_init();
   }
   if (warp == 2) {
@@ -534,9 +528,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
         const uint64_t r = f2_add(rs2[0], rs2[1]);
         l += f2_lo(r) + f2_hi(r);
       }
-      if (rescale_o) {
-        // O holds every P V up to the previous tile (completed before S of
-        // this tile was signalled); the next P V is issued after p_full
+      // O holds every P V up to the previous tile (completed before S of this
+      // tile was signalled); the next P V is issued after p_full.  The
+      // tensor-memory accesses are warp-collective: the whole warp takes the
+      // branch when any of its rows rescales (alpha = 1 on the others).
+      if (!rescale_o) alpha = 1.f;
+      if (__any_sync(0xffffffffu, rescale_o)) {
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t o[32];
@@ -568,7 +565,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
         if (p.lse != nullptr && qrow < p.n)
           p.lse[(static_cast<long long>(qt.b) * p.H + qt.h) * p.n + qrow] = (m + __log2f(l)) * 0.69314718055994531f;
       } else {
-        // tail chunk: park the unnormalised row, then the last chunk merges
+        // tail chunk: park the unnormalised rows; for each warp's 32 rows the
+        // chunk that finishes last merges every chunk's rows (a ticket per
+        // (tail, warp): no thread waits for another warp)
         const int K = p.tail_chunks;
         const long long slot = static_cast<long long>(un.tail) * K + un.chunk;
         float4* po = reinterpret_cast<float4*>(p.part_o + (slot * kBM + row) * kHeadDim);
@@ -584,40 +583,64 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
         p.part_ml[(slot * 2 + 0) * kBM + row] = m;
         p.part_ml[(slot * 2 + 1) * kBM + row] = l;
         __threadfence();
-        named_sync(1, kBM);
-        if (row == 0) bars.merge = (atomicAdd(&p.tail_ticket[un.tail], 1u) == static_cast<unsigned>(K - 1)) ? 1 : 0;
-        named_sync(1, kBM);
-        if (bars.merge) {
+        __syncwarp();
+        unsigned* ticket = p.tail_ticket + static_cast<long long>(un.tail) * 4 + quarter;
+        unsigned last = 0;
+        if (lane == 0) last = (atomicAdd(ticket, 1u) == static_cast<unsigned>(K - 1)) ? 1u : 0u;
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
           __threadfence();
           const long long base = static_cast<long long>(un.tail) * K;
+          // this thread's row: the chunks' weights 2^(m_c - M) and the total
+          // row sum L, in chunk order
+          float wc[kAttendMaxChunksPerTail];
           float M = -INFINITY;
-          for (int c = 0; c < K; ++c) M = fmaxf(M, __ldcg(p.part_ml + ((base + c) * 2) * kBM + row));
+#pragma unroll
+          for (int c = 0; c < kAttendMaxChunksPerTail; ++c) {
+            wc[c] = c < K ? __ldcg(p.part_ml + ((base + c) * 2) * kBM + row) : -INFINITY;
+            M = fmaxf(M, wc[c]);
+          }
           float L = 0.f;
-          float acc[kHeadDim];
 #pragma unroll
-          for (int d = 0; d < kHeadDim; ++d) acc[d] = 0.f;
-          for (int c = 0; c < K; ++c) {
-            const float mc = __ldcg(p.part_ml + ((base + c) * 2) * kBM + row);
-            const float w = ex2_approx(mc - M);
-            L += w * __ldcg(p.part_ml + ((base + c) * 2 + 1) * kBM + row);
-            const float4* src = reinterpret_cast<const float4*>(p.part_o + ((base + c) * kBM + row) * kHeadDim);
-#pragma unroll
-            for (int v = 0; v < kHeadDim / 4; ++v) {
-              const float4 x = __ldcg(src + v);
-              acc[4 * v + 0] = fmaf(w, x.x, acc[4 * v + 0]);
-              acc[4 * v + 1] = fmaf(w, x.y, acc[4 * v + 1]);
-              acc[4 * v + 2] = fmaf(w, x.z, acc[4 * v + 2]);
-              acc[4 * v + 3] = fmaf(w, x.w, acc[4 * v + 3]);
+          for (int c = 0; c < kAttendMaxChunksPerTail; ++c) {
+            if (c < K) {
+              wc[c] = ex2_approx(wc[c] - M);
+              L += wc[c] * __ldcg(p.part_ml + ((base + c) * 2 + 1) * kBM + row);
+            } else {
+              wc[c] = 0.f;
             }
           }
-          if (qrow < p.n) {
-            const float inv = 1.f / L;
+          if (p.lse != nullptr && qrow < p.n)
+            p.lse[(static_cast<long long>(qt.b) * p.H + qt.h) * p.n + qrow] = (M + __log2f(L)) * 0.69314718055994531f;
+          const float invL = 1.f / L;
+          // the warp's 32 rows one at a time, lane l owning dims 4l .. 4l+3:
+          // each chunk's row is one coalesced 512-byte read
+          const int r0 = quarter * 32;
+#pragma unroll 2
+          for (int r = 0; r < 32; ++r) {
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) store_row_bf16(dst + cc * 4, acc + 32 * cc, inv);
-            if (p.lse != nullptr)
-              p.lse[(static_cast<long long>(qt.b) * p.H + qt.h) * p.n + qrow] = (M + __log2f(L)) * 0.69314718055994531f;
+            for (int c = 0; c < kAttendMaxChunksPerTail; ++c) {
+              const float w = __shfl_sync(0xffffffffu, wc[c], r);
+              if (c < K) {
+                const float4 x =
+                    __ldcg(reinterpret_cast<const float4*>(p.part_o + ((base + c) * kBM + r0 + r) * kHeadDim) + lane);
+                acc.x = fmaf(w, x.x, acc.x);
+                acc.y = fmaf(w, x.y, acc.y);
+                acc.z = fmaf(w, x.z, acc.z);
+                acc.w = fmaf(w, x.w, acc.w);
+              }
+            }
+            const float inv = __shfl_sync(0xffffffffu, invL, r);
+            const int qr = qt.qt * kBM + r0 + r;
+            if (qr < p.n) {
+              uint2 v;
+              v.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+              v.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+              reinterpret_cast<uint2*>(O + ((static_cast<long long>(qt.b) * p.n + qr) * p.H + qt.h) * kHeadDim)[lane] = v;
+            }
           }
-          if (row == 0) p.tail_ticket[un.tail] = 0u;   // ready for the next launch
+          if (lane == 0) *ticket = 0u;   // ready for the next launch
         }
       }
     }

@@ -209,7 +209,7 @@ struct AttendParams {
   int tail_chunks;      // context chunks each ragged last query tile is split into (1 = not split)
   float* part_o;        // [tails * tail_chunks, 128, 128] unnormalised partial outputs
   float* part_ml;       // [tails * tail_chunks, 2, 128] partial row max / row sum
-  unsigned* tail_ticket;  // [tails], zero on entry, left zero on exit
+  unsigned* tail_ticket;  // [tails, 4] per (tail, warp of 32 rows); zero on entry, left zero on exit
   int rotate_sink;      // 1: rotate the sink keys' temporal pairs by sink_rope as they are loaded
   RopeTable sink_rope;  // e^{i theta_k total_shift}
   float scale_log2;     // log2(e) / sqrt(D)
@@ -218,12 +218,13 @@ struct AttendParams {
 };
 
 // Scratch for split tails, in the cache arena: kAttendMaxTailSlots chunk
-// slots of partial outputs and row statistics, and one ticket per tail.
+// slots of partial outputs and row statistics, and one ticket per (tail,
+// warp of 32 rows).
 constexpr int kAttendMaxTailSlots = 256;
 constexpr int kAttendMaxChunksPerTail = 8;
 constexpr size_t kAttendPartOBytes = size_t(kAttendMaxTailSlots) * 128 * 128 * 4;
 constexpr size_t kAttendPartMLBytes = size_t(kAttendMaxTailSlots) * 2 * 128 * 4;
-constexpr size_t kAttendTicketBytes = size_t(kAttendMaxTailSlots) * 4;
+constexpr size_t kAttendTicketBytes = size_t(kAttendMaxTailSlots) * 4 * 4;
 int attend_tail_chunks(int B, int H, int q_tiles, int n_tiles);
 
 cudaError_t launch_attend(const AttendParams& p, cudaStream_t st);

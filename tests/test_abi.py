@@ -67,8 +67,8 @@ def test_cache_bytes_layout(pf):
                  + al((1 + slabs) * 4)      # batch and slab tickets
                  + al(slots * 1536 * 4))    # mean key of every pool slot
     # shared attention scratch: 256 split-tail slots of 128x128 fp32 partial
-    # outputs, their row max / row sum, and 256 tickets
-    scratch = 256 * 128 * 128 * 4 + 256 * 2 * 128 * 4 + 256 * 4
+    # outputs, their row max / row sum, and a ticket per (tail, 32-row warp)
+    scratch = 256 * 128 * 128 * 4 + 256 * 2 * 128 * 4 + 256 * 4 * 4
     assert got == 256 + scratch + per_layer
     # layers scale linearly
     c.layers = 30
