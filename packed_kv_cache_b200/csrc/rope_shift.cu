@@ -8,12 +8,14 @@
 //
 // HBM-bound: per key vector and head we read and write the first
 // ceil(2*pairs/8) 16-byte words (6 words = 96 bytes for 22 pairs, three
-// 32-byte sectors each way).  One thread per key vector, two vectors per
-// step with all loads issued before any math; the grid is exactly the CTAs
-// that fit on the GPU at once (no partial last wave).  (A TMA-pipelined
-// form -- 96-byte-wide boxes of 128 rows through a ring of shared-memory
-// stages, stored back by TMA -- measured 40-50 % slower on the same
-// workloads, whatever the L2 promotion and CTAs per SM.)
+// 32-byte sectors each way).  Each lane owns one word of one row-head:
+// neighbouring lanes hold a row's words, so one warp load reads 32 / NW
+// rows' contiguous pieces with every sector fully used; four steps' loads
+// are in flight before any math, and the grid is at most the CTAs that fit
+// on the GPU at once.  (One thread per row-head, which made each warp load
+// touch 32 rows through half-used sectors, measured 17 % slower; a
+// TMA-pipelined form -- 96-byte-wide boxes of 128 rows through a ring of
+// shared-memory stages, stored back by TMA -- 40-50 % slower.)
 #include <cuda_bf16.h>
 
 #include "pf_internal.h"
@@ -24,31 +26,43 @@ namespace {
 
 template <int NW>
 __global__ void __launch_bounds__(256) rope_shift_kernel(const RowRuns runs, const RopeTable tab) {
-  const long long total = runs.start[runs.n];
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  int seg = 0;
-  // two key vectors per thread per step: all twelve loads in flight before any math
-  for (long long i0 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < total; i0 += 2 * stride) {
-    uint4 w[2][NW];
-    uint4* ptr[2] = {nullptr, nullptr};
+  // lane -> (row, word): a warp covers kRows rows per step, each row's NW
+  // words read by NW neighbouring lanes (one contiguous 16 NW-byte piece per
+  // row); kU steps' loads are in flight before any arithmetic
+  constexpr int kRows = 32 / NW;
+  constexpr int kU = 4;
+  const int lane = threadIdx.x & 31;
+  if (lane >= kRows * NW) return;   // no warp-collective operations below
+  const int r_in = lane / NW, k = lane - r_in * NW;
+  float cs[4], sn[4];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const long long i = i0 + u * stride;
+  for (int q = 0; q < 4; ++q) {
+    cs[q] = tab.c[(k * 4 + q) & 31];
+    sn[q] = tab.s[(k * 4 + q) & 31];
+  }
+  const long long total = runs.start[runs.n];
+  const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long step = (static_cast<long long>(gridDim.x) * blockDim.x >> 5) * (kRows * kU);
+  int seg = 0;
+  for (long long r0 = warp * (kRows * kU); r0 < total; r0 += step) {
+    uint4 w[kU];
+    uint4* ptr[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const long long i = r0 + u * kRows + r_in;
+      ptr[u] = nullptr;
       if (i < total) {
         while (i >= runs.start[seg + 1]) ++seg;
         while (i < runs.start[seg]) --seg;
-        ptr[u] = reinterpret_cast<uint4*>(static_cast<char*>(runs.ptr[seg]) + (i - runs.start[seg]) * (kHeadDim * 2));
-#pragma unroll
-        for (int k = 0; k < NW; ++k) w[u][k] = ptr[u][k];
+        ptr[u] = reinterpret_cast<uint4*>(static_cast<char*>(runs.ptr[seg]) + (i - runs.start[seg]) * (kHeadDim * 2)) + k;
+        w[u] = *ptr[u];
       }
     }
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < kU; ++u) {
       if (ptr[u] != nullptr) {
-#pragma unroll
-        for (int k = 0; k < NW; ++k) rope_rotate_word(w[u][k], k, tab);
-#pragma unroll
-        for (int k = 0; k < NW; ++k) ptr[u][k] = w[u][k];
+        rope_rotate_word_cs(w[u], k, tab.pairs, cs, sn);
+        *ptr[u] = w[u];
       }
     }
   }
@@ -61,7 +75,8 @@ cudaError_t launch_nw(const RowRuns& runs, const RopeTable& tab, cudaStream_t st
   cudaError_t e = cap.get(&grid_cap, [](int dev, int* v) { return one_wave_grid(rope_shift_kernel<NW>, dev, v); });
   if (e != cudaSuccess) return e;
   const long long total = runs.start[runs.n];
-  const long long want = (total + 511) / 512;
+  const long long rows_per_cta = 8LL * (32 / NW) * 4;   // 8 warps, kRows rows, kU steps
+  const long long want = (total + rows_per_cta - 1) / rows_per_cta;
   const int grid = static_cast<int>(want < grid_cap ? want : grid_cap);
   rope_shift_kernel<NW><<<grid, 256, 0, st>>>(runs, tab);
   return cudaGetLastError();
