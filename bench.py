@@ -49,9 +49,10 @@ sys.path.insert(0, ROOT)
 
 WORKLOAD = "layer"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# library kernels per step besides the selection's: attend, copy_runs + kmean
-# (append with a compressed copy); rope_shift is added when a block was evicted
-LAUNCHES_PER_STEP_BASE = 3
+# library kernels per step besides the selection's and the attention's:
+# copy_runs + kmean (append with a compressed copy); rope_shift is added when
+# a block was evicted
+LAUNCHES_PER_STEP_BASE = 2
 
 
 # ---------------------------------------------------------------- distributed plumbing
@@ -450,14 +451,16 @@ def measure_block(pf, synth, dev, flush, stream, peaks, src, blocks=3) -> dict:
 
     block()
     ms = timed_ms(block, blocks, flush, stream)
+    att_launches = pf.attend_launches(cache.cfg, cache.info(0), torch.cuda.get_device_properties(dev).multi_processor_count)
     Lk = cache.info(0)["context_tokens"]
     flops = L * S * attention_flops(B, H, n, Lk, D)
     cache.poll_device_error()
     r = {"ms_per_block": round(ms, 3), "layer_step_ms": round(ms / (L * S), 4), "context_tokens": Lk,
          "attention_flop_per_block": flops,
-         # attend per layer and step; the selection's two kernels per layer at
-         # step 0; copy + key mean per layer's append; one shift launch for all sinks
-         "launches_per_block": L * S + 2 * L + 2 * L + 1,
+         # attend (and its tail merge) per layer and step; the selection's two
+         # kernels per layer at step 0; copy + key mean per layer's append; one
+         # shift launch for all sinks
+         "launches_per_block": L * S * att_launches + 2 * L + 2 * L + 1,
          "attend_block": roofline("attend_kernel (whole block: selection, appends and shifts included)", "tensor",
                                   flops, ms, peaks, src, sustained=True)}
     del cache, Qs, Ks, Vs, Kcs, O, blk
@@ -518,6 +521,9 @@ def run_gpu(args):
     Vcn = synth.bf16_normal((B, nc, H, D), seed + 2, dev)
     O = torch.empty_like(Q)
     info0 = cache.info(0)
+    # the pool is full at every step (each append evicts one block): the
+    # attention's launch count is the same for every step
+    att_launches = pf.attend_launches(cache.cfg, info0, torch.cuda.get_device_properties(dev).multi_processor_count)
     Lk = info0["context_tokens"]
     flops = attention_flops(B, H, n, Lk, D)              # this rank's heads
     # [B, live blocks] partial (then summed) block scores of the sharded selection;
@@ -546,7 +552,7 @@ def run_gpu(args):
         ev = cache.append_block(0, k, v, kc, vc)
         if ev:
             cache.rope_shift(0, pf.PART_SINK, ev * wl.block_frames)
-        return LAUNCHES_PER_STEP_BASE + nl + (1 if ev else 0)
+        return LAUNCHES_PER_STEP_BASE + nl + att_launches + (1 if ev else 0)
 
     clocks = ClockSampler(local)
     clocks.start()

@@ -275,10 +275,28 @@ pf_status pf_rope_shift(pf_cache* cache, int layer, unsigned parts, int delta, v
  * scaled scores, natural log.  Mid blocks: the stored selection if valid;
  * if the pool holds at most n_top blocks, all of them; otherwise
  * PF_ERR_STATE (call pf_select_mid first).  One kernel launch (tcgen05
- * tensor cores, TMA loads through the partitions in place).
+ * tensor cores, TMA loads through the partitions in place), and a second
+ * (the merge of the ragged last query tiles' context chunks, launched as a
+ * programmatic dependent) when the block has an odd number of 128-row query
+ * tiles and pf_attend_tail_plan gives more than one chunk.
  */
 pf_status pf_attend(pf_cache* cache, int layer, const void* Q, const void* K_cur,
                     const void* V_cur, void* O, float* lse, void* stream);
+
+/*
+ * How pf_attend cuts the ragged last 128-row query tile of every (batch
+ * item, head) along the context when a block has an odd number of query
+ * tiles.  Pure host arithmetic (no device, no cache): with `full_units`
+ * pairs of full query tiles and `tails` ragged tiles, each over `n_tiles`
+ * 128-key tiles, on a GPU with `sms` SMs, the first *big chunks cover key
+ * tiles [0, *split) in equal parts (sized so that the SMs the last wave of
+ * pairs leaves idle finish them alongside it) and the next *small chunks
+ * cover [*split, n_tiles) (about one per SM).  *big + *small == 1 means the
+ * tiles are not split.  PF_ERR_ARG on a negative size, sms < 1 or a null
+ * output.
+ */
+pf_status pf_attend_tail_plan(long long full_units, int tails, int n_tiles, int sms, int* big, int* small,
+                              int* split);
 
 /*
  * One layer's attention at one denoising step of the current block
@@ -288,8 +306,8 @@ pf_status pf_attend(pf_cache* cache, int layer, const void* Q, const void* K_cur
  * step's queries, then pf_attend; step > 0: pf_attend with the selection
  * stored at step 0 (PF_ERR_STATE if the pool changed since, or if no
  * selection was made while the pool holds more than n_top blocks).
- * Arguments as for pf_attend; step >= 0.  Three kernel launches at step 0
- * (selection, attention), one after.
+ * Arguments as for pf_attend; step >= 0.  The selection's two kernel
+ * launches at step 0, then pf_attend's.
  */
 pf_status pf_attend_step(pf_cache* cache, int layer, int step, const void* Q, const void* K_cur,
                          const void* V_cur, void* O, float* lse, void* stream);

@@ -115,6 +115,8 @@ def _load():
         "pf_select_mid_ex": ([vp, i32, vp, ctypes.POINTER(SelectOpts), vp, vp, vp], i32),
         "pf_rope_shift": ([vp, i32, u32, i32, vp], i32),
         "pf_attend": ([vp, i32, vp, vp, vp, vp, vp, vp], i32),
+        "pf_attend_tail_plan": ([ctypes.c_longlong, i32, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32),
+                                 ctypes.POINTER(i32)], i32),
         "pf_poll_device_error": ([vp, vp, ctypes.POINTER(u32)], i32),
         "pf_selftest_wait_timeout": ([vp, u32, vp], i32),
         "pf_select_mid_static": ([vp, i32, i32, i32, vp, i32, i32, i32, i32, i32, vp, vp, vp], i32),
@@ -278,6 +280,30 @@ def pf_attend(handle, layer, Q, K_cur, V_cur, O, lse=None, stream=None) -> None:
     "Bounded Attention Context"), into O; optional natural-log LSE."""
     _check("pf_attend", lib.pf_attend(handle, layer, _dev(Q, "Q"), _dev(K_cur, "K_cur"), _dev(V_cur, "V_cur"),
                                       _dev(O, "O"), _dev(lse, "lse"), _stream(stream)))
+
+
+def pf_attend_tail_plan(full_units: int, tails: int, n_tiles: int, sms: int) -> tuple:
+    """(big, small, split): how pf_attend cuts the ragged last query tiles
+    along the context (host arithmetic only)."""
+    big, small, split = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    _check("pf_attend_tail_plan", lib.pf_attend_tail_plan(full_units, tails, n_tiles, sms, ctypes.byref(big),
+                                                          ctypes.byref(small), ctypes.byref(split)))
+    return big.value, small.value, split.value
+
+
+def attend_launches(cfg, info: dict, sms: int) -> int:
+    """Kernels one pf_attend call launches for a layer in state `info`
+    (pf_cache_layer_info) on a GPU with `sms` SMs."""
+    n = cfg.block_frames * cfg.h * cfg.w
+    q_tiles = (n + 127) // 128
+    if q_tiles % 2 == 0:
+        return 1
+    sb = lambda rows: (rows + 31) // 32  # noqa: E731
+    n_c = (cfg.block_frames // 2) * (cfg.h // 4) * (cfg.w // 4)   # tokens of a compressed block
+    n_sub = sb(info["sink_filled"] * n) + info["n_selected"] * sb(n_c) + info["recent_count"] * sb(n) + sb(n)
+    n_tiles = (n_sub + 3) // 4
+    big, small, _ = pf_attend_tail_plan(cfg.batch * cfg.heads * (q_tiles // 2), cfg.batch * cfg.heads, n_tiles, sms)
+    return 1 if big + small == 1 else 2
 
 
 def pf_attend_step(handle, layer, step, Q, K_cur, V_cur, O, lse=None, stream=None) -> None:

@@ -11,11 +11,14 @@
 //  * full unit: two 128-row query tiles of one (batch item, head) that share
 //    every K/V tile of the context;
 //  * tail chunk: when a block has an odd number of 128-row query tiles, the
-//    last (ragged) tile of each (b, h) is split along the context into k
+//    last (ragged) tile of each (b, h) is split along the context into
 //    chunks of K/V tiles.  Each chunk writes its unnormalised output, row
 //    maximum and row sum to scratch; the chunk that finishes last merges them
 //    (O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c).  The chunks run after
-//    the full units and fill what would otherwise be a nearly idle last wave.
+//    the full units: first big chunks, sized so that the SMs the last wave of
+//    full units leaves idle finish them alongside it, then small chunks,
+//    about one per SM, so that the launch ends within a few K/V tiles of
+//    the last full unit.
 // 12 warps per CTA:
 //   warp 0      TMA producer: Q, then K and V tiles through rings
 //   warp 1      MMA issuer (one thread): S_t = Q_t K^T and O_t += P_t V
@@ -155,8 +158,8 @@ __device__ __forceinline__ int subbox_valid(const AttendParams& p, int s, float 
 }
 
 // The unit of this CTA.  Units 0 .. F-1 are full units ((b, h) major, then
-// query-tile pair); then, if q_tiles is odd, B*H*tail_chunks tail chunks
-// ((b, h) major, then chunk).
+// query-tile pair); then, if q_tiles is odd, the B*H*tail_big big tail
+// chunks ((b, h) major, then chunk), then the B*H*tail_small small ones.
 struct QTile {
   int b, h, qt;
 };
@@ -183,12 +186,25 @@ __device__ __forceinline__ Unit unit_of(const AttendParams& p, int u) {
     r.chunk = 0;
   } else {
     const int v = u - F;
-    const int bh = v / p.tail_chunks, c = v - bh * p.tail_chunks;
+    const int nb = p.B * p.H * p.tail_big;
+    int bh, c;
+    if (v < nb) {
+      bh = v / p.tail_big;
+      c = v - bh * p.tail_big;
+      r.j0 = static_cast<int>(static_cast<long long>(c) * p.tail_split / p.tail_big);
+      r.j1 = static_cast<int>(static_cast<long long>(c + 1) * p.tail_split / p.tail_big);
+    } else {
+      const int v2 = v - nb;
+      bh = v2 / p.tail_small;
+      const int cs = v2 - bh * p.tail_small;
+      const int rest = p.n_tiles - p.tail_split;
+      r.j0 = p.tail_split + static_cast<int>(static_cast<long long>(cs) * rest / p.tail_small);
+      r.j1 = p.tail_split + static_cast<int>(static_cast<long long>(cs + 1) * rest / p.tail_small);
+      c = p.tail_big + cs;
+    }
     r.t[0] = {bh / p.H, bh % p.H, p.q_tiles - 1};
     r.t[1] = r.t[0];
     r.nq = 1;
-    r.j0 = static_cast<int>(static_cast<long long>(c) * p.n_tiles / p.tail_chunks);
-    r.j1 = static_cast<int>(static_cast<long long>(c + 1) * p.n_tiles / p.tail_chunks);
     r.tail = (p.tail_chunks > 1) ? bh : -1;
     r.chunk = c;
   }
@@ -241,6 +257,9 @@ __device__ __forceinline__ void store_row_bf16(uint4* dst, const float* o, float
 }
 
 __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_constant__ AttendParams p) {
+  // tail_merge_kernel (a programmatic dependent) may be scheduled once every
+  // CTA has started; it waits for this grid's completion before reading
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars& bars = *reinterpret_cast<Bars*>(smem + kOffBar);
@@ -565,11 +584,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
         if (p.lse != nullptr && qrow < p.n)
           p.lse[(static_cast<long long>(qt.b) * p.H + qt.h) * p.n + qrow] = (m + __log2f(l)) * 0.69314718055994531f;
       } else {
-        // tail chunk: park the unnormalised rows; for each warp's 32 rows the
-        // chunk that finishes last merges every chunk's rows (a ticket per
-        // (tail, warp): no thread waits for another warp)
-        const int K = p.tail_chunks;
-        const long long slot = static_cast<long long>(un.tail) * K + un.chunk;
+        // tail chunk: park the unnormalised rows; tail_merge_kernel merges
+        // the chunks once the whole grid is done
+        const long long slot = static_cast<long long>(un.tail) * p.tail_chunks + un.chunk;
         float4* po = reinterpret_cast<float4*>(p.part_o + (slot * kBM + row) * kHeadDim);
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
@@ -582,66 +599,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
         }
         p.part_ml[(slot * 2 + 0) * kBM + row] = m;
         p.part_ml[(slot * 2 + 1) * kBM + row] = l;
-        __threadfence();
-        __syncwarp();
-        unsigned* ticket = p.tail_ticket + static_cast<long long>(un.tail) * 4 + quarter;
-        unsigned last = 0;
-        if (lane == 0) last = (atomicAdd(ticket, 1u) == static_cast<unsigned>(K - 1)) ? 1u : 0u;
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
-          __threadfence();
-          const long long base = static_cast<long long>(un.tail) * K;
-          // this thread's row: the chunks' weights 2^(m_c - M) and the total
-          // row sum L, in chunk order
-          float wc[kAttendMaxChunksPerTail];
-          float M = -INFINITY;
-#pragma unroll
-          for (int c = 0; c < kAttendMaxChunksPerTail; ++c) {
-            wc[c] = c < K ? __ldcg(p.part_ml + ((base + c) * 2) * kBM + row) : -INFINITY;
-            M = fmaxf(M, wc[c]);
-          }
-          float L = 0.f;
-#pragma unroll
-          for (int c = 0; c < kAttendMaxChunksPerTail; ++c) {
-            if (c < K) {
-              wc[c] = ex2_approx(wc[c] - M);
-              L += wc[c] * __ldcg(p.part_ml + ((base + c) * 2 + 1) * kBM + row);
-            } else {
-              wc[c] = 0.f;
-            }
-          }
-          if (p.lse != nullptr && qrow < p.n)
-            p.lse[(static_cast<long long>(qt.b) * p.H + qt.h) * p.n + qrow] = (M + __log2f(L)) * 0.69314718055994531f;
-          const float invL = 1.f / L;
-          // the warp's 32 rows one at a time, lane l owning dims 4l .. 4l+3:
-          // each chunk's row is one coalesced 512-byte read
-          const int r0 = quarter * 32;
-#pragma unroll 2
-          for (int r = 0; r < 32; ++r) {
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int c = 0; c < kAttendMaxChunksPerTail; ++c) {
-              const float w = __shfl_sync(0xffffffffu, wc[c], r);
-              if (c < K) {
-                const float4 x =
-                    __ldcg(reinterpret_cast<const float4*>(p.part_o + ((base + c) * kBM + r0 + r) * kHeadDim) + lane);
-                acc.x = fmaf(w, x.x, acc.x);
-                acc.y = fmaf(w, x.y, acc.y);
-                acc.z = fmaf(w, x.z, acc.z);
-                acc.w = fmaf(w, x.w, acc.w);
-              }
-            }
-            const float inv = __shfl_sync(0xffffffffu, invL, r);
-            const int qr = qt.qt * kBM + r0 + r;
-            if (qr < p.n) {
-              uint2 v;
-              v.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-              v.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-              reinterpret_cast<uint2*>(O + ((static_cast<long long>(qt.b) * p.n + qr) * p.H + qt.h) * kHeadDim)[lane] = v;
-            }
-          }
-          if (lane == 0) *ticket = 0u;   // ready for the next launch
-        }
       }
     }
   }
@@ -652,6 +609,58 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
     __syncwarp();   // the allocating warp may have run the rotator loop
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// The split ragged tiles' merge: CTA (tail, g) finishes rows 16 g .. 16 g + 15
+// of tail (b, h)'s last query tile from its chunks' partial outputs,
+// O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c, M = max_c m_c.  Warp w
+// takes rows 2w and 2w + 1; for a row, lane c holds chunk c's statistics and
+// lane l dims 4l .. 4l + 3, every chunk's piece of the row in flight at once.
+__global__ void __launch_bounds__(256) tail_merge_kernel(const __grid_constant__ AttendParams p) {
+  // the attention grid's partial outputs: complete and visible after this
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int tail = blockIdx.x;
+  const int K = p.tail_chunks;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = tail / p.H, h = tail - b * p.H;
+  const long long base = static_cast<long long>(tail) * K;
+  __nv_bfloat16* O = static_cast<__nv_bfloat16*>(p.O);
+  for (int rr = 0; rr < 2; ++rr) {
+    const int row = blockIdx.y * 16 + warp * 2 + rr;
+    const int qrow = (p.q_tiles - 1) * kBM + row;
+    if (qrow >= p.n) continue;   // the same for the whole warp
+    const float mc = lane < K ? __ldcg(p.part_ml + ((base + lane) * 2) * kBM + row) : -INFINITY;
+    const float lc = lane < K ? __ldcg(p.part_ml + ((base + lane) * 2 + 1) * kBM + row) : 0.f;
+    float4 x[kAttendMaxChunksPerTail];
+#pragma unroll
+    for (int c = 0; c < kAttendMaxChunksPerTail; ++c)
+      if (c < K) x[c] = __ldcg(reinterpret_cast<const float4*>(p.part_o + ((base + c) * kBM + row) * kHeadDim) + lane);
+    float M = mc;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float w = lane < K ? ex2_approx(mc - M) : 0.f;
+    float L = w * lc;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int c = 0; c < kAttendMaxChunksPerTail; ++c) {
+      const float wc = __shfl_sync(0xffffffffu, w, c);
+      if (c < K) {
+        acc.x = fmaf(wc, x[c].x, acc.x);
+        acc.y = fmaf(wc, x[c].y, acc.y);
+        acc.z = fmaf(wc, x[c].z, acc.z);
+        acc.w = fmaf(wc, x[c].w, acc.w);
+      }
+    }
+    const float inv = 1.f / L;
+    uint2 v;
+    v.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    v.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    reinterpret_cast<uint2*>(O + ((static_cast<long long>(b) * p.n + qrow) * p.H + h) * kHeadDim)[lane] = v;
+    if (lane == 0 && p.lse != nullptr)
+      p.lse[(static_cast<long long>(b) * p.H + h) * p.n + qrow] = (M + __log2f(L)) * 0.69314718055994531f;
   }
 }
 
@@ -672,28 +681,78 @@ __global__ void wait_timeout_kernel(unsigned* err, long long lim) {
 
 }  // namespace
 
-int attend_tail_chunks(int B, int H, int q_tiles, int n_tiles) {
-  if ((q_tiles & 1) == 0) return 1;
-  const int tails = B * H;
-  int k = kAttendMaxTailSlots / tails;
-  if (k > kAttendMaxChunksPerTail) k = kAttendMaxChunksPerTail;
-  if (k > n_tiles) k = n_tiles;
-  return k < 1 ? 1 : k;
+TailPlan attend_tail_plan(long long F, int T, int n, int sms) {
+  const TailPlan whole{1, 0, n};
+  if (T <= 0 || n <= 0 || sms <= 0) return whole;
+  int max_k = kAttendMaxTailSlots / T;
+  if (max_k > kAttendMaxChunksPerTail) max_k = kAttendMaxChunksPerTail;
+  if (max_k > n) max_k = n;
+  if (max_k <= 1) return whole;
+  const int per_sm = static_cast<int>((2LL * sms + T) / (2LL * T));   // round(sms / T): ~one small chunk per SM
+  const int small_all = per_sm < 1 ? 1 : (per_sm > max_k ? max_k : per_sm);
+  if (F <= 0) return TailPlan{0, small_all, 0};
+  const long long waves = (F + sms - 1) / sms;
+  const long long idle = sms - (F - (waves - 1) * sms);   // SMs the last wave of full units leaves idle
+  if (idle <= 0) return TailPlan{0, small_all, 0};
+  // big work per tail: what the idle SMs do during one full unit's time
+  const int J = static_cast<int>(idle * n / T < n ? idle * n / T : n);
+  int kb = 0;
+  for (int k = 1; k < max_k && k <= J; ++k) {
+    // the T k big chunks, ceil(T k / idle) per idle SM, fit in n K/V tiles
+    if ((T * static_cast<long long>(k) + idle - 1) / idle * ((J + k - 1) / k) <= n) {
+      kb = k;
+      break;
+    }
+  }
+  if (kb == 0) return TailPlan{max_k, 0, n};
+  const int rest = n - J;
+  int ks = 0;
+  if (rest > 0) {
+    ks = per_sm;
+    if (ks > max_k - kb) ks = max_k - kb;
+    if (ks > rest) ks = rest;
+    if (ks < 1) ks = 1;
+  }
+  return TailPlan{kb, ks, J};
 }
 
 cudaError_t launch_attend(const AttendParams& p, cudaStream_t st) {
-  // the kernel's shared-memory limit is raised once per device
-  static PerDevice attr;
-  int unused = 0;
-  cudaError_t e = attr.get(&unused, [](int, int*) {
-    return cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  // once per device: the kernel's shared-memory limit is raised and the SM
+  // count read
+  static PerDevice sms_of;
+  int sms = 0;
+  cudaError_t e = sms_of.get(&sms, [](int dev, int* v) {
+    cudaError_t r = cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (r != cudaSuccess) return r;
+    return cudaDeviceGetAttribute(v, cudaDevAttrMultiProcessorCount, dev);
   });
   if (e != cudaSuccess) return e;
+  AttendParams q = p;
   const long long bh = 1LL * p.B * p.H;
-  const long long units = bh * (p.q_tiles / 2) + ((p.q_tiles & 1) ? bh * p.tail_chunks : 0);
+  const long long F = bh * (p.q_tiles / 2);
+  const TailPlan tp = (p.q_tiles & 1) ? attend_tail_plan(F, static_cast<int>(bh), p.n_tiles, sms)
+                                      : TailPlan{1, 0, p.n_tiles};
+  q.tail_big = tp.big;
+  q.tail_small = tp.small;
+  q.tail_split = tp.split;
+  q.tail_chunks = tp.big + tp.small;
+  const long long units = F + ((p.q_tiles & 1) ? bh * q.tail_chunks : 0);
   if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
-  attend_kernel<<<static_cast<unsigned>(units), kThreads, kSmemBytes, st>>>(p);
-  return cudaGetLastError();
+  attend_kernel<<<static_cast<unsigned>(units), kThreads, kSmemBytes, st>>>(q);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || !(p.q_tiles & 1) || q.tail_chunks <= 1) return e;
+  // the split ragged tiles' merge, a programmatic dependent of the attention grid
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(bh), kBM / 16);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tail_merge_kernel, q);
 }
 
 cudaError_t launch_wait_timeout_selftest(unsigned* err, long long lim, cudaStream_t st) {

@@ -48,7 +48,7 @@ constexpr int kMaxPoolSlots = 8192;                         // the top-k keeps a
 
 // attention scratch shared by all layers: split-tail partial outputs, row
 // statistics and tickets
-constexpr size_t kAttendScratchBytes = pf::kAttendPartOBytes + pf::kAttendPartMLBytes + pf::kAttendTicketBytes;
+constexpr size_t kAttendScratchBytes = pf::kAttendPartOBytes + pf::kAttendPartMLBytes;
 
 struct Geometry {
   int n, n_c, slots, HD;
@@ -223,7 +223,6 @@ struct pf_cache {
   unsigned* err;  // device error word
   float* part_o;
   float* part_ml;
-  unsigned* tail_ticket;
   long long timeout_cycles;
   std::vector<Layer> L;
 };
@@ -366,7 +365,6 @@ pf_status pf_cache_create(const pf_config* cfg, void* dev_arena, size_t arena_by
   char* p = c->arena + kAlign;
   c->part_o = reinterpret_cast<float*>(p); p += pf::kAttendPartOBytes;
   c->part_ml = reinterpret_cast<float*>(p); p += pf::kAttendPartMLBytes;
-  c->tail_ticket = reinterpret_cast<unsigned*>(p); p += pf::kAttendTicketBytes;
   for (int l = 0; l < cfg->layers; ++l) {
     Layer& Ly = c->L[l];
     const Geometry& g = c->g;
@@ -771,6 +769,17 @@ pf_status pf_rope_shift(pf_cache* c, int layer, unsigned parts, int delta, void*
   return PF_OK;
 }
 
+pf_status pf_attend_tail_plan(long long full_units, int tails, int n_tiles, int sms, int* big, int* small,
+                              int* split) {
+  if (big == nullptr || small == nullptr || split == nullptr) return fail(PF_ERR_ARG, "null output");
+  if (full_units < 0 || tails < 0 || n_tiles < 0 || sms < 1) return fail(PF_ERR_ARG, "negative size or sms < 1");
+  const pf::TailPlan tp = pf::attend_tail_plan(full_units, tails, n_tiles, sms);
+  *big = tp.big;
+  *small = tp.small;
+  *split = tp.split;
+  return PF_OK;
+}
+
 pf_status pf_attend(pf_cache* c, int layer, const void* Q, const void* K_cur, const void* V_cur, void* O, float* lse,
                     void* stream) {
   pf_status s = check_layer(c, layer);
@@ -849,10 +858,8 @@ pf_status pf_attend(pf_cache* c, int layer, const void* Q, const void* K_cur, co
   p.sb_mid_hi = p.sb_sink + n_sel * p.sb_mid;
   p.exact = (sink_rows % 32 == 0 && g.n % 32 == 0) ? 1 : 0;
   p.q_tiles = (g.n + 127) / 128;
-  p.tail_chunks = pf::attend_tail_chunks(B, H, p.q_tiles, p.n_tiles);
   p.part_o = c->part_o;
   p.part_ml = c->part_ml;
-  p.tail_ticket = c->tail_ticket;
   p.rotate_sink = (cf.sink_rope_in_attention && Ly.total_shift != 0 && sink_rows > 0) ? 1 : 0;
   p.sink_rope.pairs = cf.rope_split[0] / 2;
   for (int k = 0; k < 32; ++k) {

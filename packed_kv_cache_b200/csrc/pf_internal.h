@@ -207,9 +207,10 @@ struct AttendParams {
                         // the padding after the last key have partial sub-boxes
   int q_tiles;          // 128-row query tiles per (b, h)
   int tail_chunks;      // context chunks each ragged last query tile is split into (1 = not split)
+  int tail_big, tail_small;  // of them: the first tail_big cover K/V tiles [0, tail_split) in equal
+  int tail_split;            // parts, the other tail_small cover [tail_split, n_tiles) (set by launch_attend)
   float* part_o;        // [tails * tail_chunks, 128, 128] unnormalised partial outputs
   float* part_ml;       // [tails * tail_chunks, 2, 128] partial row max / row sum
-  unsigned* tail_ticket;  // [tails, 4] per (tail, warp of 32 rows); zero on entry, left zero on exit
   int rotate_sink;      // 1: rotate the sink keys' temporal pairs by sink_rope as they are loaded
   RopeTable sink_rope;  // e^{i theta_k total_shift}
   float scale_log2;     // log2(e) / sqrt(D)
@@ -218,14 +219,19 @@ struct AttendParams {
 };
 
 // Scratch for split tails, in the cache arena: kAttendMaxTailSlots chunk
-// slots of partial outputs and row statistics, and one ticket per (tail,
-// warp of 32 rows).
+// slots of partial outputs and row statistics.
 constexpr int kAttendMaxTailSlots = 256;
-constexpr int kAttendMaxChunksPerTail = 8;
+constexpr int kAttendMaxChunksPerTail = 16;
 constexpr size_t kAttendPartOBytes = size_t(kAttendMaxTailSlots) * 128 * 128 * 4;
 constexpr size_t kAttendPartMLBytes = size_t(kAttendMaxTailSlots) * 2 * 128 * 4;
-constexpr size_t kAttendTicketBytes = size_t(kAttendMaxTailSlots) * 4 * 4;
-int attend_tail_chunks(int B, int H, int q_tiles, int n_tiles);
+// How the T ragged tiles of a launch are cut along the context (n K/V tiles
+// each), given F full units and `sms` SMs: big chunks that the SMs left idle
+// by the last wave of full units finish alongside it, then about one small
+// chunk per SM for the rest.  {big, small, split}.
+struct TailPlan {
+  int big, small, split;
+};
+TailPlan attend_tail_plan(long long F, int T, int n, int sms);
 
 cudaError_t launch_attend(const AttendParams& p, cudaStream_t st);
 

@@ -67,8 +67,8 @@ def test_cache_bytes_layout(pf):
                  + al((1 + slabs) * 4)      # batch and slab tickets
                  + al(slots * 1536 * 4))    # mean key of every pool slot
     # shared attention scratch: 256 split-tail slots of 128x128 fp32 partial
-    # outputs, their row max / row sum, and a ticket per (tail, 32-row warp)
-    scratch = 256 * 128 * 128 * 4 + 256 * 2 * 128 * 4 + 256 * 4 * 4
+    # outputs and their row max / row sum
+    scratch = 256 * 128 * 128 * 4 + 256 * 2 * 128 * 4
     assert got == 256 + scratch + per_layer
     # layers scale linearly
     c.layers = 30
@@ -338,19 +338,19 @@ def _c_kind(decl: str) -> str:
     words = decl.replace("const", "").split()
     base = " ".join(words[:-1]) if len(words) > 1 else words[0]
     return {"int": "int", "pf_status": "int", "unsigned": "unsigned", "unsigned int": "unsigned",
-            "size_t": "size_t", "float": "float"}[base]
+            "size_t": "size_t", "float": "float", "long long": "long long"}[base]
 
 
 def _ctypes_kind(t) -> str:
     if t in (ctypes.c_void_p, ctypes.c_char_p) or hasattr(t, "_type_") and isinstance(t._type_, type):
         return "pointer"
     return {ctypes.c_int: "int", ctypes.c_uint: "unsigned", ctypes.c_size_t: "size_t",
-            ctypes.c_float: "float"}[t]
+            ctypes.c_float: "float", ctypes.c_longlong: "long long"}[t]
 
 
 def test_binding_argtypes_match_the_prototypes(pf):
     # each declared function: the same number of parameters, each of the same
-    # kind (pointer, int, unsigned, size_t, float), and the same result kind
+    # kind (pointer, int, unsigned, size_t, long long, float), and the same result kind
     text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
     protos = re.findall(r"([A-Za-z_][\w ]*?\**)\s*\b(pf_[a-z_0-9]+)\s*\(([^)]*)\)\s*;", text)
     assert len(protos) == len(declared_functions())
@@ -373,3 +373,29 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     r = subprocess.run([sys.executable, "-c", "import packed_kv_cache_b200"], cwd=tmp_path,
                        capture_output=True, text=True)
     assert r.returncode != 0 and "libpf.so" in r.stderr
+
+
+def test_attend_tail_plan(pf):
+    # the pages-scale layer on 148 SMs: 288 pairs leave 8 SMs idle in the
+    # last wave; each of the 12 ragged tiles gets two 73-tile chunks for them
+    # and 12 small chunks for the end (about one per SM)
+    assert pf.pf_attend_tail_plan(288, 12, 219, 148) == (2, 12, 146)
+    assert pf.pf_attend_tail_plan(576, 24, 219, 148) == (2, 6, 146)
+    # no ragged tiles, or one key tile: nothing to split
+    assert pf.pf_attend_tail_plan(288, 0, 219, 148) == (1, 0, 219)
+    assert pf.pf_attend_tail_plan(288, 12, 1, 148) == (1, 0, 1)
+    # more tails than scratch slots for two chunks each: not split
+    assert pf.pf_attend_tail_plan(0, 200, 100, 148) == (1, 0, 100)
+    import random
+    rng = random.Random(5)
+    for _ in range(3000):
+        F, T, n, sms = rng.randint(0, 3000), rng.randint(1, 300), rng.randint(1, 6000), rng.choice([1, 7, 148, 160])
+        big, small, split = pf.pf_attend_tail_plan(F, T, n, sms)
+        K = big + small
+        assert 1 <= K <= 16 and (K == 1 or T * K <= 256)
+        bounds = [c * split // big for c in range(big)] + [split + c * (n - split) // small for c in range(small)]
+        bounds.append(n)
+        assert bounds[0] == 0 and all(a < b for a, b in zip(bounds, bounds[1:]))   # every chunk has key tiles
+    for bad in ((-1, 1, 1, 1), (1, -1, 1, 1), (1, 1, -1, 1), (1, 1, 1, 0)):
+        with pytest.raises(pf.PFError):
+            pf.pf_attend_tail_plan(*bad)
