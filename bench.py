@@ -392,7 +392,7 @@ def measure_stress(pf, synth, dev, flush, stream, peaks, src, iters) -> dict:
         O = torch.empty_like(d["Q"])
         Lk = cache.info(0)["context_tokens"]
         ms = timed_ms(lambda: cache.attend(0, d["Q"], d["K_cur"], d["V_cur"], O), iters, flush, stream)
-        r["attend"] = roofline("attend_kernel", "tensor", attention_flops(B, H, n, Lk, D), ms, peaks, src)
+        r["attend"] = roofline("attend_kernel + tail_merge_kernel", "tensor", attention_flops(B, H, n, Lk, D), ms, peaks, src)
         r["context_tokens"] = Lk
         cache.poll_device_error()
         out[name] = r
@@ -411,7 +411,7 @@ def measure_dense(pf, synth, dev, flush, stream, peaks, src, iters) -> dict:
     Lk = cache.info(0)["context_tokens"]
     ms = timed_ms(lambda: cache.attend(0, d["Q"], d["K_cur"], d["V_cur"], O), iters, flush, stream)
     r = {"context_tokens": Lk,
-         "attend": roofline("attend_kernel", "tensor", attention_flops(wl.batch, wl.heads, wl.n, Lk), ms, peaks, src)}
+         "attend": roofline("attend_kernel + tail_merge_kernel", "tensor", attention_flops(wl.batch, wl.heads, wl.n, Lk), ms, peaks, src)}
     cache.poll_device_error()
     del cache, d, O
     torch.cuda.empty_cache()
@@ -461,7 +461,7 @@ def measure_block(pf, synth, dev, flush, stream, peaks, src, blocks=3) -> dict:
          # kernels per layer at step 0; copy + key mean per layer's append; one
          # shift launch for all sinks
          "launches_per_block": L * S * att_launches + 2 * L + 2 * L + 1,
-         "attend_block": roofline("attend_kernel (whole block: selection, appends and shifts included)", "tensor",
+         "attend_block": roofline("attend_kernel + tail_merge_kernel (whole block: selection, appends and shifts included)", "tensor",
                                   flops, ms, peaks, src, sustained=True)}
     del cache, Qs, Ks, Vs, Kcs, O, blk
     torch.cuda.empty_cache()
@@ -663,7 +663,7 @@ def run_gpu(args):
         configs = measure_configs(which, pf, synth, dev, flush, stream, peaks, peak_src, max(args.steps, 5))
     t_run1 = time.time()
     clocks.stop()
-    att = roofline("attend_kernel", "tensor", flops, att_mean_ms, peaks, peak_src,
+    att = roofline("attend_kernel + tail_merge_kernel", "tensor", flops, att_mean_ms, peaks, peak_src,
                    traffic=traffic_for(os.path.join(ROOT, "packed_kv_cache_b200", "csrc", "attend.cu"), WORKLOAD))
     line = {
         "metric": "packed-cache attention TFLOP/s (per-layer step)",
