@@ -168,26 +168,37 @@ __device__ void select_tail(const SelectArgs& a, int b, uint32_t* keys) {
 }
 
 // keys[0 .. count) hold the block scores' sort keys (scores already written).
+// Radix select on 8-bit digits of the keys, most significant first: each
+// pass counts the digits of the keys that still match the prefix (warp-
+// aggregated shared-memory atomics), then warp 0 scans the 256 counts and
+// picks the digit holding the need-th largest key.  Two block barriers per
+// pass (the next pass's histogram is cleared during this one).  Then one
+// block scan of the packed (above-threshold, equal) counts gives every
+// thread's first output position: selected blocks are the keys above the
+// threshold T and the `need` oldest equal to it, written in ascending age.
 __device__ void select_topk_from_keys(const SelectArgs& a, int b, uint32_t* keys) {
-  __shared__ unsigned hist[256];
+  __shared__ unsigned hist[2][256];
   __shared__ unsigned sh_prefix, sh_need;
-  const int t = threadIdx.x;
+  static_assert(kThreads == 256, "one histogram bin per thread");
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int count = a.count;
   if (!a.topk) {   // scores only
     if (t == 0) a.ticket[b] = 0u;
     return;
   }
   const int k_sel = min(a.n_top, count);
+  const bool take_all = (k_sel == count);
+  hist[0][t] = 0u;
+  hist[1][t] = 0u;
   if (t == 0) {
     sh_prefix = 0u;
     sh_need = static_cast<unsigned>(k_sel);
   }
   __syncthreads();
-  const bool take_all = (k_sel == count);
   if (!take_all) {
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      hist[t] = 0u;
-      __syncthreads();
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      unsigned* h = hist[pass & 1];
       const unsigned pre = sh_prefix;
       // warp-aggregated: one shared-memory atomic per distinct digit per warp
       // (the keys' leading digits are mostly equal)
@@ -199,20 +210,34 @@ __device__ void select_topk_from_keys(const SelectArgs& a, int b, uint32_t* keys
         const unsigned m = __ballot_sync(0xffffffffu, take);
         if (take) {
           const unsigned grp = __match_any_sync(m, digit);
-          if ((t & 31) == __ffs(grp) - 1) atomicAdd(&hist[digit], static_cast<unsigned>(__popc(grp)));
+          if (lane == __ffs(grp) - 1) atomicAdd(&h[digit], static_cast<unsigned>(__popc(grp)));
         }
       }
+      hist[(pass + 1) & 1][t] = 0u;   // the next pass's histogram (last read two barriers ago)
       __syncthreads();
-      {
-        // suffix sums over the digits, from 255 down: thread t holds digit 255 - t
-        const unsigned hc = hist[255 - t];
-        unsigned tot;
-        const unsigned before = block_exclusive_scan(hc, &tot);   // count of digits > 255 - t
+      if (warp == 0) {
+        // lane l: digits 255 - 8 l - i, i = 0..7 (descending over the warp)
+        unsigned c[8], sum = 0u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          c[i] = h[255 - 8 * lane - i];
+          sum += c[i];
+        }
+        unsigned incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        unsigned before = incl - sum;   // keys whose digit is above this lane's digits
         const unsigned need = sh_need;
-        __syncthreads();
-        if (before < need && before + hc >= need) {               // exactly one thread
-          sh_prefix = pre | (static_cast<unsigned>(255 - t) << shift);
-          sh_need = need - before;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (before < need && before + c[i] >= need) {   // exactly one (lane, i)
+            sh_prefix = pre | (static_cast<unsigned>(255 - 8 * lane - i) << shift);
+            sh_need = need - before;
+          }
+          before += c[i];
         }
       }
       __syncthreads();
@@ -222,19 +247,18 @@ __device__ void select_topk_from_keys(const SelectArgs& a, int b, uint32_t* keys
   const unsigned need = sh_need;
   const int per = (count + kThreads - 1) / kThreads;
   const int lo = min(count, t * per), hi = min(count, lo + per);
-  // rank of each key equal to the threshold among the equal ones, by age
-  unsigned eqc = 0u, tot = 0u;
-  if (!take_all)
-    for (int q = lo; q < hi; ++q) eqc += (keys[q] == T) ? 1u : 0u;
-  const unsigned eq_before = block_exclusive_scan(eqc, &tot);
-  unsigned nsel = 0u, e = eq_before;
+  unsigned gt = 0u, eq = 0u;
   for (int q = lo; q < hi; ++q) {
     const uint32_t key = keys[q];
-    const bool s = take_all || key > T || (key == T && e++ < need);
-    nsel += s ? 1u : 0u;
+    if (take_all || key > T) ++gt;
+    else if (key == T) ++eq;
   }
-  unsigned pos = block_exclusive_scan(nsel, &tot);
-  e = eq_before;
+  unsigned tot;
+  // counts <= 8,192 each: 16 bits apiece
+  const unsigned packed = block_exclusive_scan((gt << 16) | eq, &tot);
+  const unsigned gt_before = packed >> 16, eq_before = packed & 0xffffu;
+  unsigned pos = gt_before + min(eq_before, need);
+  unsigned e = eq_before;
   for (int q = lo; q < hi; ++q) {
     const uint32_t key = keys[q];
     const bool s = take_all || key > T || (key == T && e++ < need);
