@@ -421,6 +421,22 @@ def test_attention_small_full(pf, name):
     _attend_and_compare(pf, wl, d)
 
 
+def test_attention_single_ragged_tile_split_and_merged(pf):
+    # one 112-row query tile per (b, h) and no query-tile pairs: the tile is
+    # cut along the context into small chunks, which park partial outputs that
+    # the merge kernel (a second launch) combines; every row against the oracle
+    wl = synth.WORKLOADS["ragged_c"].replace(name="ragged_one", h=4, w=7, n=112, n_c=2)
+    assert wl.block_frames * wl.h * wl.w == wl.n and (wl.n + 127) // 128 == 1
+    sb = lambda rows: (rows + 31) // 32  # noqa: E731
+    n_tiles = (sb(wl.sink_blocks * wl.n) + min(wl.n_top, wl.pool_blocks) * sb(wl.n_c) + wl.recent_blocks * sb(wl.n)
+               + sb(wl.n) + 3) // 4
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    big, small, _ = pf.pf_attend_tail_plan(0, wl.batch * wl.heads, n_tiles, sms)
+    assert big + small > 1
+    d = synth.make_layer(wl, seed_for("ragged_c") + 7)
+    _attend_and_compare(pf, wl, d)
+
+
 def test_attention_split_tail_repeated_calls(pf):
     # the split-tail scratch (partial outputs, tickets) is reused across calls
     wl, d = _layer("ragged_c")
