@@ -157,9 +157,10 @@ __device__ __forceinline__ int subbox_valid(const AttendParams& p, int s, float 
   return 0;
 }
 
-// The unit of this CTA.  Units 0 .. F-1 are full units ((b, h) major, then
-// query-tile pair); then, if q_tiles is odd, the B*H*tail_big big tail
-// chunks ((b, h) major, then chunk), then the B*H*tail_small small ones.
+// The unit of this CTA.  The (b, h) are taken in groups of group_bh; a
+// group's units are its full units ((b, h) major, then query-tile pair), then
+// its ragged tiles' tail_big big chunks ((b, h) major, then chunk); after
+// every group, the B*H*tail_small small chunks ((b, h) major, then chunk).
 struct QTile {
   int b, h, qt;
 };
@@ -173,10 +174,19 @@ struct Unit {
 
 __device__ __forceinline__ Unit unit_of(const AttendParams& p, int u) {
   const int pairs = p.q_tiles / 2;
-  const int F = p.B * p.H * pairs;
+  const int BH = p.B * p.H;
+  const int kb = (p.q_tiles & 1) ? p.tail_big : 0;
+  const int per_group = p.group_bh * (pairs + kb);
+  const int grouped = BH * (pairs + kb);   // every group's pairs and big chunks
   Unit r;
-  if (u < F) {
-    const int bh = u / pairs, kk = u - bh * pairs;
+  int g = 0, rem = 0, gh = 0;
+  if (u < grouped) {
+    g = u / per_group;
+    rem = u - g * per_group;
+    gh = min(p.group_bh, BH - g * p.group_bh);
+  }
+  if (u < grouped && rem < gh * pairs) {
+    const int bh = g * p.group_bh + rem / pairs, kk = rem % pairs;
     r.t[0] = {bh / p.H, bh % p.H, 2 * kk};
     r.t[1] = {bh / p.H, bh % p.H, 2 * kk + 1};
     r.nq = 2;
@@ -185,16 +195,15 @@ __device__ __forceinline__ Unit unit_of(const AttendParams& p, int u) {
     r.tail = -1;
     r.chunk = 0;
   } else {
-    const int v = u - F;
-    const int nb = p.B * p.H * p.tail_big;
     int bh, c;
-    if (v < nb) {
-      bh = v / p.tail_big;
-      c = v - bh * p.tail_big;
+    if (u < grouped) {
+      const int v = rem - gh * pairs;
+      bh = g * p.group_bh + v / kb;
+      c = v - (v / kb) * kb;
       r.j0 = static_cast<int>(static_cast<long long>(c) * p.tail_split / p.tail_big);
       r.j1 = static_cast<int>(static_cast<long long>(c + 1) * p.tail_split / p.tail_big);
     } else {
-      const int v2 = v - nb;
+      const int v2 = u - grouped;
       bh = v2 / p.tail_small;
       const int cs = v2 - bh * p.tail_small;
       const int rest = p.n_tiles - p.tail_split;
@@ -682,29 +691,37 @@ __global__ void wait_timeout_kernel(unsigned* err, long long lim) {
 }  // namespace
 
 TailPlan attend_tail_plan(long long F, int T, int n, int sms) {
-  const TailPlan whole{1, 0, n};
-  if (T <= 0 || n <= 0 || sms <= 0) return whole;
+  if (T <= 0 || n <= 0 || sms <= 0) return TailPlan{1, 0, n, T > 0 ? T : 1};
+  // the groups of (b, h): as many as one wave's pairs take
+  const long long P = F / T;
+  long long group = P > 0 ? sms / P : T;
+  if (group < 1) group = 1;
+  if (group > T) group = T;
+  const int Tg = static_cast<int>(group);
+  const TailPlan whole{1, 0, n, Tg};
   int max_k = kAttendMaxTailSlots / T;
   if (max_k > kAttendMaxChunksPerTail) max_k = kAttendMaxChunksPerTail;
   if (max_k > n) max_k = n;
   if (max_k <= 1) return whole;
   const int per_sm = static_cast<int>((2LL * sms + T) / (2LL * T));   // round(sms / T): ~one small chunk per SM
   const int small_all = per_sm < 1 ? 1 : (per_sm > max_k ? max_k : per_sm);
-  if (F <= 0) return TailPlan{0, small_all, 0};
-  const long long waves = (F + sms - 1) / sms;
-  const long long idle = sms - (F - (waves - 1) * sms);   // SMs the last wave of full units leaves idle
-  if (idle <= 0) return TailPlan{0, small_all, 0};
+  if (F <= 0) return TailPlan{0, small_all, 0, Tg};
+  // a group's pairs, in waves; the SMs its last wave leaves idle
+  const long long Fg = group * P;
+  const long long waves = (Fg + sms - 1) / sms;
+  const long long idle = sms - (Fg - (waves - 1) * sms);
+  if (idle <= 0) return TailPlan{0, small_all, 0, Tg};
   // big work per tail: what the idle SMs do during one full unit's time
-  const int J = static_cast<int>(idle * n / T < n ? idle * n / T : n);
+  const int J = static_cast<int>(idle * n / group < n ? idle * n / group : n);
   int kb = 0;
   for (int k = 1; k < max_k && k <= J; ++k) {
     // the T k big chunks, ceil(T k / idle) per idle SM, fit in n K/V tiles
-    if ((T * static_cast<long long>(k) + idle - 1) / idle * ((J + k - 1) / k) <= n) {
+    if ((group * k + idle - 1) / idle * ((J + k - 1) / k) <= n) {
       kb = k;
       break;
     }
   }
-  if (kb == 0) return TailPlan{max_k, 0, n};
+  if (kb == 0) return TailPlan{max_k, 0, n, Tg};
   const int rest = n - J;
   int ks = 0;
   if (rest > 0) {
@@ -713,7 +730,7 @@ TailPlan attend_tail_plan(long long F, int T, int n, int sms) {
     if (ks > rest) ks = rest;
     if (ks < 1) ks = 1;
   }
-  return TailPlan{kb, ks, J};
+  return TailPlan{kb, ks, J, Tg};
 }
 
 cudaError_t launch_attend(const AttendParams& p, cudaStream_t st) {
@@ -731,10 +748,11 @@ cudaError_t launch_attend(const AttendParams& p, cudaStream_t st) {
   const long long bh = 1LL * p.B * p.H;
   const long long F = bh * (p.q_tiles / 2);
   const TailPlan tp = (p.q_tiles & 1) ? attend_tail_plan(F, static_cast<int>(bh), p.n_tiles, sms)
-                                      : TailPlan{1, 0, p.n_tiles};
+                                      : TailPlan{1, 0, p.n_tiles, static_cast<int>(bh)};
   q.tail_big = tp.big;
   q.tail_small = tp.small;
   q.tail_split = tp.split;
+  q.group_bh = tp.group;
   q.tail_chunks = tp.big + tp.small;
   const long long units = F + ((p.q_tiles & 1) ? bh * q.tail_chunks : 0);
   if (units > 0x7fffffffLL) return cudaErrorInvalidValue;

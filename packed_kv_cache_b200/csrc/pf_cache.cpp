@@ -773,7 +773,7 @@ pf_status pf_attend_tail_plan(long long full_units, int tails, int n_tiles, int 
                               int* split) {
   if (big == nullptr || small == nullptr || split == nullptr) return fail(PF_ERR_ARG, "null output");
   if (full_units < 0 || tails < 0 || n_tiles < 0 || sms < 1) return fail(PF_ERR_ARG, "negative size or sms < 1");
-  const pf::TailPlan tp = pf::attend_tail_plan(full_units, tails, n_tiles, sms);
+  const pf::TailPlan tp = pf::attend_tail_plan(full_units, tails, n_tiles, sms);   // tp.group stays internal
   *big = tp.big;
   *small = tp.small;
   *split = tp.split;

@@ -209,6 +209,7 @@ struct AttendParams {
   int tail_chunks;      // context chunks each ragged last query tile is split into (1 = not split)
   int tail_big, tail_small;  // of them: the first tail_big cover K/V tiles [0, tail_split) in equal
   int tail_split;            // parts, the other tail_small cover [tail_split, n_tiles) (set by launch_attend)
+  int group_bh;              // (b, h) per unit group: their pairs, then their tiles' big chunks
   float* part_o;        // [tails * tail_chunks, 128, 128] unnormalised partial outputs
   float* part_ml;       // [tails * tail_chunks, 2, 128] partial row max / row sum
   int rotate_sink;      // 1: rotate the sink keys' temporal pairs by sink_rope as they are loaded
@@ -225,11 +226,14 @@ constexpr int kAttendMaxChunksPerTail = 16;
 constexpr size_t kAttendPartOBytes = size_t(kAttendMaxTailSlots) * 128 * 128 * 4;
 constexpr size_t kAttendPartMLBytes = size_t(kAttendMaxTailSlots) * 2 * 128 * 4;
 // How the T ragged tiles of a launch are cut along the context (n K/V tiles
-// each), given F full units and `sms` SMs: big chunks that the SMs left idle
-// by the last wave of full units finish alongside it, then about one small
-// chunk per SM for the rest.  {big, small, split}.
+// each), given F = T P full units (P query-tile pairs per (b, h)) and `sms`
+// SMs.  The (b, h) are grouped, as many as a wave's pairs take (group =
+// sms / P), so that a group's ragged tiles are read alongside its pairs:
+// big chunks that the SMs a group's pairs leave idle finish alongside them,
+// then about one small chunk per SM for the rest.  {big, small, split, group}.
 struct TailPlan {
   int big, small, split;
+  int group;   // (b, h) whose query-tile pairs and big tail chunks are ordered together
 };
 TailPlan attend_tail_plan(long long F, int T, int n, int sms);
 
