@@ -339,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 5) score_kernel(const SelectArgs a) 
 // the chunk's rows go to qsum[b, chunk]; the chunk that finishes last (slab
 // ticket) adds the R chunk sums in chunk order into qtot[b] and clears the
 // ticket.
-constexpr int kSelLoads = 16;   // row loads in flight per thread
+constexpr int kSelLoads = 8;   // row loads in flight per thread
 template <int kGroups>
 __global__ void __launch_bounds__(kThreads, 2) qsum_slab_kernel(const SelectArgs a) {
   // let the scoring kernel be scheduled now: it waits for this grid's
