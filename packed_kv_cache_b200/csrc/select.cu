@@ -15,9 +15,10 @@
 // its rows; the last chunk of a slab adds the chunks in a fixed order), and
 // score_cached_kernel, launched as a programmatic dependent so that it
 // fetches the mean keys while the sums are formed, takes one dot product per
-// block (a warp each) and, in the last CTA of a batch item (ticket), runs an
-// exact radix select of the n_top largest scores (ties to the older block),
-// writes the selection in ascending age, and clears its ticket.  The
+// block (a warp each) and, in the last CTA of a batch item (ticket), selects
+// the n_top largest scores exactly (ties to the older block: warp sorting
+// networks for n_top <= 32, a radix select above), writes the selection in
+// ascending age, and clears its ticket.  The
 // allocation-free entry point has no cached means and streams the keys:
 //   1. qpool: the columns of Q[b] summed over the block's rows into qsum[b].
 //   2. score: one CTA per 32-row chunk of a pool block, a dot product with
@@ -142,7 +143,7 @@ __device__ unsigned block_exclusive_scan(unsigned v, unsigned* total) {
 }
 
 // The last CTA of batch item b: block scores from the partial sums, exact
-// radix selection of the n_top largest (ties to the older block), outputs in
+// selection of the n_top largest (ties to the older block), outputs in
 // ascending age, and the cleanup that leaves ticket[b] zero.
 __device__ void select_topk_from_keys(const SelectArgs& a, int b, uint32_t* keys);
 
@@ -167,6 +168,101 @@ __device__ void select_tail(const SelectArgs& a, int b, uint32_t* keys) {
   select_topk_from_keys(a, b, keys);
 }
 
+// ---- top-k of at most 32: warp-level bitonic networks ----
+// A block's rank value packs its sort key above (2^32 - 1 - q), so larger is
+// preferred: a higher score, then the older block (smaller q).  The values
+// are distinct, so the k largest are exactly the radix select's choice.
+
+__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int j) {
+  const uint32_t lo = __shfl_xor_sync(0xffffffffu, static_cast<uint32_t>(v), j);
+  const uint32_t hi = __shfl_xor_sync(0xffffffffu, static_cast<uint32_t>(v >> 32), j);
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
+__device__ __forceinline__ uint64_t shfl_u64(uint64_t v, int src) {
+  const uint32_t lo = __shfl_sync(0xffffffffu, static_cast<uint32_t>(v), src);
+  const uint32_t hi = __shfl_sync(0xffffffffu, static_cast<uint32_t>(v >> 32), src);
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
+// Four independent warp lists (one value per lane each) sorted descending
+// over the lanes (lane 0 the largest).  Bitonic network, stage (k, j): lane
+// and lane ^ j compare; the lower lane keeps the larger value where
+// (lane & k) == 0 (a descending run), the smaller elsewhere.
+__device__ __forceinline__ void warp_sort4_desc(uint64_t* v, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const bool keep_max = ((lane & j) == 0) == ((lane & k) == 0);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint64_t o = shfl_xor_u64(v[u], j);
+        v[u] = keep_max ? (v[u] > o ? v[u] : o) : (v[u] < o ? v[u] : o);
+      }
+    }
+  }
+}
+
+// The 32 largest of two descending warp lists, descending: the lane-wise
+// maximum of x and y reversed holds them as a bitonic sequence, which five
+// half-cleaner stages sort.
+__device__ __forceinline__ uint64_t warp_merge_desc(uint64_t x, uint64_t y, int lane) {
+  const uint64_t yr = shfl_u64(y, 31 - lane);
+  uint64_t m = x > yr ? x : yr;
+#pragma unroll
+  for (int j = 16; j > 0; j >>= 1) {
+    const uint64_t o = shfl_xor_u64(m, j);
+    m = ((lane & j) == 0) ? (m > o ? m : o) : (m < o ? m : o);
+  }
+  return m;
+}
+
+// The k_sel <= 32 largest of keys[0 .. count), written in ascending age.
+// Each warp folds its 32-key batches (four at a time, sorted side by side)
+// into its running 32 largest; warp 0 merges the eight warps' lists, and
+// each of the winners finds its output position by counting the winners
+// older than it.
+__device__ void select_topk_warp(const SelectArgs& a, int b, const uint32_t* keys, int k_sel) {
+  __shared__ uint64_t lists[kThreads / 32][32];
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int count = a.count;
+  __syncthreads();   // keys[] was written by every thread
+  uint64_t best = 0ull;   // 0 ranks below every real block
+  for (int qb = warp * 32; qb < count; qb += 4 * kThreads) {   // warp-uniform
+    uint64_t v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int q = qb + u * kThreads + lane;
+      v[u] = q < count ? (static_cast<uint64_t>(keys[q]) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(q)) : 0ull;
+    }
+    warp_sort4_desc(v, lane);
+    const uint64_t m = warp_merge_desc(warp_merge_desc(v[0], v[1], lane), warp_merge_desc(v[2], v[3], lane), lane);
+    best = warp_merge_desc(best, m, lane);
+  }
+  lists[warp][lane] = best;
+  __syncthreads();
+  if (warp == 0) {
+    uint64_t l[kThreads / 32];
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) l[w] = lists[w][lane];
+    const uint64_t m0 = warp_merge_desc(l[0], l[1], lane), m1 = warp_merge_desc(l[2], l[3], lane);
+    const uint64_t m2 = warp_merge_desc(l[4], l[5], lane), m3 = warp_merge_desc(l[6], l[7], lane);
+    const uint64_t top = warp_merge_desc(warp_merge_desc(m0, m1, lane), warp_merge_desc(m2, m3, lane), lane);
+    const uint32_t q = 0xFFFFFFFFu - static_cast<uint32_t>(top);
+    int pos = 0;
+#pragma unroll
+    for (int s = 0; s < 32; ++s) {
+      const uint32_t qs = __shfl_sync(0xffffffffu, q, s);
+      pos += (s < k_sel && qs < q) ? 1 : 0;
+    }
+    if (lane < k_sel) {
+      a.sel_slots[static_cast<long long>(b) * a.n_top + pos] = (a.head + static_cast<int>(q)) % a.slots;
+      if (a.sel_out) a.sel_out[static_cast<long long>(b) * k_sel + pos] = static_cast<int>(q);
+    }
+  }
+}
+
 // keys[0 .. count) hold the block scores' sort keys (scores already written).
 // Radix select on 8-bit digits of the keys, most significant first: each
 // pass counts the digits of the keys that still match the prefix (warp-
@@ -188,6 +284,11 @@ __device__ void select_topk_from_keys(const SelectArgs& a, int b, uint32_t* keys
   }
   const int k_sel = min(a.n_top, count);
   const bool take_all = (k_sel == count);
+  if (!take_all && k_sel <= 32) {
+    select_topk_warp(a, b, keys, k_sel);
+    if (t == 0) a.ticket[b] = 0u;
+    return;
+  }
   hist[0][t] = 0u;
   hist[1][t] = 0u;
   if (t == 0) {

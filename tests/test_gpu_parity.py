@@ -334,6 +334,25 @@ def test_head_shard_scores_sum_then_given_top_k(pf):
     assert torch.equal(O_g, O_full)
 
 
+@pytest.mark.parametrize("P,k", [(33, 1), (33, 32), (34, 33), (40, 16), (257, 32), (300, 17), (1000, 16),
+                                 (1025, 32), (1025, 64), (3000, 5), (8191, 32)])
+def test_given_scores_top_k(pf, P, k):
+    # the top-k on its own, through given scores: up to 32 blocks by warp
+    # sorting networks, more by the radix select.  Five distinct values (the
+    # choice is mostly the older-block tie rule), then distinct scores.
+    wl = _wl("tiny").replace(batch=2, pool_blocks=P, mid_capacity=P, n_top=k, planted=0)
+    d = synth.make_layer(wl, 7)
+    cache = build_cache(pf, wl, d)
+    assert cache.info(0)["mid_count"] == P
+    rng = np.random.default_rng(P * 97 + k)
+    for scores in (rng.integers(-2, 3, size=(wl.batch, P)).astype(np.float32),
+                   rng.standard_normal((wl.batch, P)).astype(np.float32)):
+        sel = torch.full((wl.batch, k), -1, dtype=torch.int32, device="cuda")
+        cache.select_mid_ex(0, policy=pf.ROUTE_GIVEN, scores_in=torch.from_numpy(scores).cuda(), sel_out=sel)
+        torch.cuda.synchronize()
+        assert np.array_equal(sel.cpu().numpy(), oracle.select_topk(scores, k))
+
+
 @pytest.mark.parametrize("name", ["ragged_b", "ragged_c"])
 def test_random_and_fifo_routing_then_attention(pf, name):
     # the pages' routing baselines: random blocks (random scores passed in)
