@@ -215,6 +215,13 @@ class ClockSampler:
             s["source"] = self.source
         return s
 
+    def window_at_least(self, t0: float, t1: float, n: int = 3):
+        """The same, widened around [t0, t1] until it holds n samples."""
+        s = summarize_rows_at_least(self.rows, t0, t1, n)
+        if s is not None:
+            s["source"] = self.source
+        return s
+
 
 REASON_BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
                "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
@@ -262,6 +269,23 @@ def summarize_rows(rows, t0: float | None = None, t1: float | None = None):
     reasons = sorted({x for r in sel for x in r[3]})
     return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
             "reasons": reasons, "samples": len(sel)}
+
+
+def summarize_rows_at_least(rows, t0: float, t1: float, n: int = 3, max_pad_s: float = 5.0):
+    """summarize_rows over [t0, t1], widened symmetrically (10 ms, doubling,
+    at most max_pad_s each side) until it holds at least n samples: a timed
+    region of a few tens of ms can fall between two samples of the host
+    thread.  The record says which window it covers ("window_s") and how far
+    past the timed region it reaches ("pad_s")."""
+    pad = 0.0
+    s = summarize_rows(rows, t0, t1)
+    while (s is None or s["samples"] < n) and pad < max_pad_s:
+        pad = min(max_pad_s, 0.01 if pad == 0.0 else 2 * pad)
+        s = summarize_rows(rows, t0 - pad, t1 + pad)
+    if s is not None:
+        s["window_s"] = round(t1 - t0 + 2 * pad, 3)
+        s["pad_s"] = pad
+    return s
 
 
 def summarize_clocks(lines, t0: float | None = None, t1: float | None = None):
@@ -694,7 +718,7 @@ def run_gpu(args):
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / args.steps, 4)},
         "gpu_launches": launches,
-        "clocks": clocks.window(t_start, t_end),
+        "clocks": clocks.window_at_least(t_start, t_end),
         "clocks_run": clocks.window(t_run0, t_run1),
         "configs": configs,
     }

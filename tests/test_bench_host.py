@@ -81,6 +81,22 @@ def test_sampled_rows_summarised_inside_the_window():
     assert bench.summarize_rows(rows, 20.0, 30.0) is None
 
 
+def test_timed_window_widened_until_it_holds_samples():
+    rows = [(9.0, 1965.0, 1965.0, []), (9.95, 1900.0, 1965.0, ["sw_power_cap"]), (10.06, 1960.0, 1965.0, []),
+            (10.2, 1950.0, 1965.0, []), (30.0, 800.0, 1965.0, ["hw_slowdown"])]
+    # a 40 ms timed region between two samples: widened 10, 20, 40, 80 ms, then 160 ms each side
+    s = bench.summarize_rows_at_least(rows, 10.0, 10.04, n=3)
+    assert s["samples"] == 3 and s["pad_s"] == 0.16 and s["window_s"] == 0.36
+    assert s["reasons"] == ["sw_power_cap"] and s["sm_mhz"] == 1950.0
+    # enough samples inside: left as it is
+    s = bench.summarize_rows_at_least(rows, 9.0, 10.2, n=3)
+    assert s["samples"] == 4 and s["pad_s"] == 0.0
+    # never past max_pad_s: the slow sample 20 s away stays out
+    s = bench.summarize_rows_at_least(rows, 10.0, 10.04, n=10, max_pad_s=5.0)
+    assert s["samples"] == 4 and s["pad_s"] == 5.0 and "hw_slowdown" not in s["reasons"]
+    assert bench.summarize_rows_at_least([], 1.0, 2.0) is None
+
+
 def test_head_shards_and_roofline_record():
     assert [bench.head_shard(12, 8, r) for r in range(8)] == [(0, 2), (2, 4), (4, 6), (6, 8), (8, 9), (9, 10),
                                                              (10, 11), (11, 12)]
