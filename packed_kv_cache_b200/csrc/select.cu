@@ -159,11 +159,31 @@ __device__ __forceinline__ void put_score(const SelectArgs& a, int b, uint32_t* 
 __device__ void select_tail(const SelectArgs& a, int b, uint32_t* keys) {
   const int t = threadIdx.x;
   const int count = a.count;
-  for (int q = t; q < count; q += kThreads) {
-    const float* pp = a.partial + static_cast<long long>(b) * a.partial_ld + static_cast<long long>(q) * a.p_stride;
-    float s = 0.f;
-    for (int k = 0; k < a.chunks_per_block; ++k) s += __ldcg(pp + static_cast<long long>(k) * a.k_stride);
-    put_score(a, b, keys, q, s);
+  const float* pb = a.partial + static_cast<long long>(b) * a.partial_ld;
+  if (a.chunks_per_block == 1) {
+    // one partial per block: a thread's next eight loaded before any score
+    // is stored (the stores could otherwise alias the next loads)
+    constexpr int kBatch = 8;
+    for (int q0 = t; q0 < count; q0 += kThreads * kBatch) {
+      float s[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int q = q0 + u * kThreads;
+        s[u] = q < count ? __ldcg(pb + static_cast<long long>(q) * a.p_stride) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int q = q0 + u * kThreads;
+        if (q < count) put_score(a, b, keys, q, 0.f + s[u]);   // 0 + s: the sum the loop below forms
+      }
+    }
+  } else {
+    for (int q = t; q < count; q += kThreads) {
+      const float* pp = pb + static_cast<long long>(q) * a.p_stride;
+      float s = 0.f;
+      for (int k = 0; k < a.chunks_per_block; ++k) s += __ldcg(pp + static_cast<long long>(k) * a.k_stride);
+      put_score(a, b, keys, q, s);
+    }
   }
   select_topk_from_keys(a, b, keys);
 }
@@ -503,16 +523,15 @@ __global__ void __launch_bounds__(kThreads, 2) qsum_slab_kernel(const SelectArgs
   if (!is_last) return;
   __threadfence();
   if (t < kCols) {
-    // the R chunk sums in chunk order, eight loads in flight
+    // the R chunk sums in chunk order, all of them in flight at once
     const float* src = a.qsum + static_cast<long long>(b) * kSelMaxRowChunks * a.HD + col0 + t;
+    float v[kSelMaxRowChunks];
+#pragma unroll
+    for (int k = 0; k < kSelMaxRowChunks; ++k) v[k] = k < R ? __ldcg(src + static_cast<long long>(k) * a.HD) : 0.f;
     float sum = 0.f;
-    for (int c0 = 0; c0 < R; c0 += 8) {
-      float v[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) v[k] = c0 + k < R ? __ldcg(src + static_cast<long long>(c0 + k) * a.HD) : 0.f;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) sum += v[k];
-    }
+    for (int k = 0; k < kSelMaxRowChunks; ++k)
+      if (k < R) sum += v[k];
     a.qtot[static_cast<long long>(b) * a.HD + col0 + t] = sum;
   }
 }
