@@ -11,8 +11,8 @@
 // 32-byte sectors each way).  Each lane owns one word of one row-head:
 // neighbouring lanes hold a row's words, so one warp load reads 32 / NW
 // rows' contiguous pieces with every sector fully used; four steps' loads
-// are in flight before any math, and the grid is at most the CTAs that fit
-// on the GPU at once.  (One thread per row-head, which made each warp load
+// are in flight before any math; the grid depends on the size (see
+// launch_nw).  (One thread per row-head, which made each warp load
 // touch 32 rows through half-used sectors, measured 17 % slower; a
 // TMA-pipelined form -- 96-byte-wide boxes of 128 rows through a ring of
 // shared-memory stages, stored back by TMA -- 40-50 % slower.)
@@ -68,6 +68,13 @@ __global__ void __launch_bounds__(256) rope_shift_kernel(const RowRuns runs, con
   }
 }
 
+// Grid: a shift of at least kUncappedWaves times the CTAs resident at once
+// (every cached key of a stress layer) gets one CTA per 8 warps' share, so
+// finished CTAs are replaced rather than looping (0.189 against 0.209 ms on
+// the batch-2 stress layer); a smaller one (the method's sink shift) loops
+// over the resident CTAs, which avoids a ragged last wave (15.4 against
+// 17.4 µs).
+constexpr long long kUncappedWaves = 8;
 template <int NW>
 cudaError_t launch_nw(const RowRuns& runs, const RopeTable& tab, cudaStream_t st) {
   static PerDevice cap;
@@ -77,8 +84,9 @@ cudaError_t launch_nw(const RowRuns& runs, const RopeTable& tab, cudaStream_t st
   const long long total = runs.start[runs.n];
   const long long rows_per_cta = 8LL * (32 / NW) * 4;   // 8 warps, kRows rows, kU steps
   const long long want = (total + rows_per_cta - 1) / rows_per_cta;
-  const int grid = static_cast<int>(want < grid_cap ? want : grid_cap);
-  rope_shift_kernel<NW><<<grid, 256, 0, st>>>(runs, tab);
+  const long long grid = want >= kUncappedWaves * grid_cap ? want : (want < grid_cap ? want : grid_cap);
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+  rope_shift_kernel<NW><<<static_cast<int>(grid), 256, 0, st>>>(runs, tab);
   return cudaGetLastError();
 }
 
