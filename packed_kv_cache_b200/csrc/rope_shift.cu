@@ -84,8 +84,8 @@ cudaError_t launch_nw(const RowRuns& runs, const RopeTable& tab, cudaStream_t st
   const long long total = runs.start[runs.n];
   const long long rows_per_cta = 8LL * (32 / NW) * 4;   // 8 warps, kRows rows, kU steps
   const long long want = (total + rows_per_cta - 1) / rows_per_cta;
-  const long long grid = want >= kUncappedWaves * grid_cap ? want : (want < grid_cap ? want : grid_cap);
-  if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+  long long grid = want >= kUncappedWaves * grid_cap ? want : (want < grid_cap ? want : grid_cap);
+  if (grid > 0x7fffffffLL) grid = 0x7fffffffLL;   // the kernel strides over whatever the grid leaves
   rope_shift_kernel<NW><<<static_cast<int>(grid), 256, 0, st>>>(runs, tab);
   return cudaGetLastError();
 }
